@@ -1,0 +1,524 @@
+// C-ABI of libengram: argument checks, workspace layout and the launch
+// sequence of each entry point declared in include/engram.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "engram_internal.cuh"
+
+namespace engram {
+
+namespace {
+
+thread_local char g_err[512] = "";
+std::atomic<uint32_t> g_debug{0};
+
+engram_status fail(engram_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+engram_status cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ENGRAM_OK;
+  return fail(ENGRAM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int max_order(const engram_config& c) {
+  int m = 0;
+  for (int i = 0; i < c.n_orders; ++i) m = c.orders[i] > m ? c.orders[i] : m;
+  return m;
+}
+
+engram_status check_config(const engram_config* c) {
+  if (c == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "config is NULL");
+  if (c->n_orders < 1 || c->n_orders > ENGRAM_MAX_ORDERS)
+    return fail(ENGRAM_ERR_INVALID_ARG, "n_orders=%d outside [1, %d]", c->n_orders, ENGRAM_MAX_ORDERS);
+  for (int i = 0; i < c->n_orders; ++i) {
+    if (c->orders[i] < 1 || c->orders[i] > ENGRAM_MAX_NGRAM)
+      return fail(ENGRAM_ERR_INVALID_ARG, "orders[%d]=%d outside [1, %d]", i, c->orders[i], ENGRAM_MAX_NGRAM);
+    if (i > 0 && c->orders[i] <= c->orders[i - 1])
+      return fail(ENGRAM_ERR_INVALID_ARG, "orders must be strictly ascending");
+  }
+  if (c->heads_per_order < 1 || c->n_orders * c->heads_per_order > ENGRAM_MAX_HEADS)
+    return fail(ENGRAM_ERR_INVALID_ARG, "n_orders*heads_per_order must be in [1, %d]", ENGRAM_MAX_HEADS);
+  if (c->row_dim < 1) return fail(ENGRAM_ERR_INVALID_ARG, "row_dim=%d < 1", c->row_dim);
+  if (c->hidden < 1) return fail(ENGRAM_ERR_INVALID_ARG, "hidden=%d < 1", c->hidden);
+  if (c->hc_mult < 1 || c->hc_mult > ENGRAM_MAX_HC)
+    return fail(ENGRAM_ERR_INVALID_ARG, "hc_mult=%d outside [1, %d]", c->hc_mult, ENGRAM_MAX_HC);
+  if (c->conv_kernel < 1 || c->conv_kernel > ENGRAM_MAX_CONV_K)
+    return fail(ENGRAM_ERR_INVALID_ARG, "conv_kernel=%d outside [1, %d]", c->conv_kernel, ENGRAM_MAX_CONV_K);
+  if (c->dilation < 1) return fail(ENGRAM_ERR_INVALID_ARG, "dilation=%d < 1", c->dilation);
+  if (c->pad_id < 0 || c->pad_id >= (int64_t(1) << 32))
+    return fail(ENGRAM_ERR_INVALID_ARG, "pad_id must be in [0, 2^32)");
+  if (c->vocab < 1 || c->vocab > (int64_t(1) << 32))
+    return fail(ENGRAM_ERR_INVALID_ARG, "vocab must be in [1, 2^32]");
+  if (!(c->rms_eps > 0.f)) return fail(ENGRAM_ERR_INVALID_ARG, "rms_eps must be > 0");
+  if (!(c->gate_eps >= 0.f)) return fail(ENGRAM_ERR_INVALID_ARG, "gate_eps must be >= 0");
+  if (c->dtype != ENGRAM_F32 && c->dtype != ENGRAM_BF16)
+    return fail(ENGRAM_ERR_INVALID_ARG, "unknown dtype %d", static_cast<int>(c->dtype));
+  return ENGRAM_OK;
+}
+
+// Shapes the projection, gate and conv kernels need.
+engram_status check_dense_shapes(const engram_config* c) {
+  if (c->hidden % 64 != 0)
+    return fail(ENGRAM_ERR_UNSUPPORTED, "hidden=%d must be a multiple of 64", c->hidden);
+  return ENGRAM_OK;
+}
+
+engram_status fill_hash_params(const engram_config* c, const int64_t* mult, const int64_t* primes,
+                               HashParams* hp) {
+  if (mult == nullptr || primes == nullptr)
+    return fail(ENGRAM_ERR_INVALID_ARG, "multipliers / primes (host arrays) must be non-NULL");
+  memset(hp, 0, sizeof *hp);
+  const int mx = max_order(*c);
+  hp->n_orders = c->n_orders;
+  hp->J = c->heads_per_order;
+  hp->nh = c->n_orders * c->heads_per_order;
+  hp->n_hist = mx - 1;
+  for (int i = 0; i < c->n_orders; ++i) hp->orders[i] = c->orders[i];
+  for (int k = 0; k < mx; ++k) {
+    // t < 2^32 and m < 2^31 keep every product, hence every xor, below 2^63
+    if (mult[k] <= 0 || mult[k] >= (int64_t(1) << 31) || (mult[k] & 1) == 0)
+      return fail(ENGRAM_ERR_INVALID_ARG, "multipliers[%d]=%lld must be odd and in (0, 2^31)", k,
+                  static_cast<long long>(mult[k]));
+    hp->mult[k] = static_cast<uint64_t>(mult[k]);
+  }
+  for (int h = 0; h < hp->nh; ++h) {
+    if (primes[h] < 2 || primes[h] >= (int64_t(1) << 31))
+      return fail(ENGRAM_ERR_INVALID_ARG, "primes[%d]=%lld outside [2, 2^31)", h,
+                  static_cast<long long>(primes[h]));
+    hp->prime[h] = static_cast<uint64_t>(primes[h]);
+    hp->barrett[h] = ~uint64_t(0) / hp->prime[h];
+  }
+  hp->vocab = c->vocab;
+  hp->pad_id = c->pad_id;
+  return ENGRAM_OK;
+}
+
+// Workspace of the projection/gate stage for M tokens (both engines).
+struct StageLayout {
+  size_t v_off, part_off, g_off, end;
+};
+StageLayout stage_layout(const engram_config* c, int64_t M, size_t start) {
+  StageLayout L;
+  const size_t es = c->dtype == ENGRAM_F32 ? 4 : 2;
+  const int n_tiles_max = c->hidden / kSimtTileN;
+  L.v_off = align256(start);
+  L.part_off = align256(L.v_off + static_cast<size_t>(M) * c->hidden * es);
+  L.g_off = align256(L.part_off + static_cast<size_t>(M) * c->hc_mult * n_tiles_max * sizeof(float4));
+  L.end = align256(L.g_off + static_cast<size_t>(M) * c->hc_mult * sizeof(float));
+  return L;
+}
+
+int64_t rows_ld(int64_t M) { return (M + 127) / 128 * 128; }
+
+struct ForwardLayout {
+  size_t rows_off;
+  StageLayout st;
+};
+ForwardLayout forward_layout(const engram_config* c, int64_t M) {
+  ForwardLayout L;
+  L.rows_off = 0;
+  const int nh = c->n_orders * c->heads_per_order;
+  L.st = stage_layout(c, M, static_cast<size_t>(nh) * rows_ld(M) * sizeof(int32_t));
+  return L;
+}
+
+bool use_tc(const engram_config* c) {
+  if (g_debug.load() & ENGRAM_DEBUG_FORCE_SIMT) return false;
+  return tc_projection_supported(c->row_dim, c->hidden, c->dtype);
+}
+
+// The projection + gate stage shared by engram_forward and engram_gate_fuse.
+engram_status run_stage(const engram_config* c, ProjParams pp, float* g, float* g_copy,
+                        cudaStream_t s) {
+  const bool tc = use_tc(c);
+  pp.n_tiles = c->hidden / (tc ? kTcTileN : kSimtTileN);
+  pp.debug = g_debug.load();
+  engram_status st = tc ? cuda_check(launch_proj_tc(pp, s), "projection (tcgen05)")
+                        : cuda_check(launch_proj_simt(pp, s), "projection (SIMT)");
+  if (st != ENGRAM_OK) return st;
+  GateParams gp;
+  gp.partials = pp.partials;
+  gp.g = g;
+  gp.g_copy = g_copy;
+  gp.M = pp.M;
+  gp.hc = c->hc_mult;
+  gp.n_tiles = pp.n_tiles;
+  gp.H = c->hidden;
+  gp.rms_eps = c->rms_eps;
+  gp.gate_eps = c->gate_eps;
+  return cuda_check(launch_gate(gp, s), "gate");
+}
+
+}  // namespace
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace engram
+
+using namespace engram;
+
+extern "C" {
+
+int32_t engram_version(void) { return 10000 * 0 + 100 * 1 + 0; }
+
+size_t engram_last_error(char* buf, size_t n) {
+  size_t len = strlen(g_err);
+  if (buf != nullptr && n > 0) {
+    size_t k = len < n - 1 ? len : n - 1;
+    memcpy(buf, g_err, k);
+    buf[k] = '\0';
+  }
+  return len;
+}
+
+void engram_set_debug(uint32_t flags) { g_debug.store(flags); }
+
+int32_t engram_projection_engine(const engram_config* cfg) {
+  if (check_config(cfg) != ENGRAM_OK) return -1;
+  return use_tc(cfg) ? ENGRAM_ENGINE_TCGEN05 : ENGRAM_ENGINE_SIMT;
+}
+
+engram_status engram_read_status(uint32_t* dev_status, uint32_t* host_bits, engram_stream stream) {
+  if (dev_status == nullptr || host_bits == nullptr)
+    return fail(ENGRAM_ERR_INVALID_ARG, "dev_status / host_bits must be non-NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  engram_status st = cuda_check(cudaMemcpyAsync(host_bits, dev_status, sizeof(uint32_t),
+                                                cudaMemcpyDeviceToHost, s), "status copy");
+  if (st != ENGRAM_OK) return st;
+  st = cuda_check(cudaMemsetAsync(dev_status, 0, sizeof(uint32_t), s), "status clear");
+  if (st != ENGRAM_OK) return st;
+  st = cuda_check(cudaStreamSynchronize(s), "stream synchronize");
+  if (st != ENGRAM_OK) return st;
+  if (*host_bits & ENGRAM_STATUS_TIMEOUT)
+    return fail(ENGRAM_ERR_TIMEOUT, "a bounded pipeline wait ran out (status 0x%x)", *host_bits);
+  if (*host_bits & (ENGRAM_STATUS_ID_RANGE | ENGRAM_STATUS_ROW_RANGE))
+    return fail(ENGRAM_ERR_ID_RANGE, "ids or rows out of range (status 0x%x)", *host_bits);
+  return ENGRAM_OK;
+}
+
+engram_status engram_compress_ids(const int64_t* raw, int64_t n, const int64_t* lookup,
+                                  int64_t raw_vocab, int64_t* out, uint32_t* dev_status,
+                                  engram_stream stream) {
+  if (n < 0) return fail(ENGRAM_ERR_INVALID_ARG, "n < 0");
+  if (n > 0 && (raw == nullptr || lookup == nullptr || out == nullptr))
+    return fail(ENGRAM_ERR_INVALID_ARG, "raw / lookup / out must be non-NULL");
+  if (raw_vocab < 1) return fail(ENGRAM_ERR_INVALID_ARG, "raw_vocab < 1");
+  return cuda_check(launch_compress(raw, n, lookup, raw_vocab, out, dev_status,
+                                    static_cast<cudaStream_t>(stream)), "compress");
+}
+
+engram_status engram_hash(const engram_config* cfg, const int64_t* ids, int32_t B, int32_t T,
+                          const int64_t* history, const int64_t* multipliers,
+                          const int64_t* primes, int64_t* idx, uint32_t* dev_status,
+                          engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
+  if (static_cast<int64_t>(B) * T > 0 && (ids == nullptr || idx == nullptr))
+    return fail(ENGRAM_ERR_INVALID_ARG, "ids / idx must be non-NULL");
+  HashParams hp;
+  st = fill_hash_params(cfg, multipliers, primes, &hp);
+  if (st != ENGRAM_OK) return st;
+  hp.ids = ids;
+  hp.history = history;
+  hp.idx_out = idx;
+  hp.status = dev_status;
+  hp.B = B;
+  hp.T = T;
+  return cuda_check(launch_hash(hp, static_cast<cudaStream_t>(stream)), "hash");
+}
+
+engram_status engram_gather(const engram_config* cfg, const void* table, int64_t total_rows,
+                            const int64_t* row_offsets, const int64_t* idx, int64_t M, void* e,
+                            uint32_t* dev_status, engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (M < 0) return fail(ENGRAM_ERR_INVALID_ARG, "M < 0");
+  if (row_offsets == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "row_offsets (host) is NULL");
+  if (M > 0 && (table == nullptr || idx == nullptr || e == nullptr))
+    return fail(ENGRAM_ERR_INVALID_ARG, "table / idx / e must be non-NULL");
+  if (total_rows < 1) return fail(ENGRAM_ERR_INVALID_ARG, "total_rows < 1");
+  GatherParams gp;
+  memset(&gp, 0, sizeof gp);
+  gp.table = table;
+  gp.idx = idx;
+  gp.e = e;
+  gp.status = dev_status;
+  gp.M = M;
+  gp.total_rows = total_rows;
+  gp.nh = cfg->n_orders * cfg->heads_per_order;
+  gp.row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
+  if (gp.row_bytes % 4 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "row bytes must be a multiple of 4");
+  if (gp.row_bytes % 16 == 0 && (!aligned16(table) || !aligned16(e)))
+    return fail(ENGRAM_ERR_INVALID_ARG, "table and e must be 16-byte aligned");
+  for (int h = 0; h < gp.nh; ++h) gp.row_off[h] = row_offsets[h];
+  return cuda_check(launch_gather(gp, static_cast<cudaStream_t>(stream)), "gather");
+}
+
+engram_status engram_gate_fuse_workspace_size(const engram_config* cfg, int64_t M, size_t* bytes) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (M < 0 || bytes == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "M < 0 or bytes NULL");
+  *bytes = stage_layout(cfg, M, 0).end;
+  return ENGRAM_OK;
+}
+
+engram_status engram_gate_fuse(const engram_config* cfg, const void* e, const void* w_value,
+                               const void* w_key, const void* norm_key, const void* norm_query,
+                               const void* hidden, int64_t M, void* u, float* gates, void* ws,
+                               size_t ws_bytes, uint32_t* dev_status, engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  st = check_dense_shapes(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (M < 0) return fail(ENGRAM_ERR_INVALID_ARG, "M < 0");
+  if (M == 0) return ENGRAM_OK;
+  const void* ptrs[] = {e, w_value, w_key, norm_key, norm_query, hidden, u, ws};
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "a tensor / workspace pointer is NULL");
+    if (!aligned16(p)) return fail(ENGRAM_ERR_INVALID_ARG, "tensor / workspace pointers must be 16-byte aligned");
+  }
+  const StageLayout L = stage_layout(cfg, M, 0);
+  if (ws_bytes < L.end)
+    return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", ws_bytes, L.end);
+  char* w = static_cast<char*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ProjParams pp;
+  memset(&pp, 0, sizeof pp);
+  pp.a_src = e;
+  pp.rows = nullptr;
+  pp.a_rows = M * cfg->n_orders * cfg->heads_per_order;
+  pp.w_value = w_value;
+  pp.w_key = w_key;
+  pp.norm_key = norm_key;
+  pp.norm_query = norm_query;
+  pp.hidden = hidden;
+  pp.V = w + L.v_off;
+  pp.partials = reinterpret_cast<float4*>(w + L.part_off);
+  pp.status = dev_status;
+  pp.M = M;
+  pp.nh = cfg->n_orders * cfg->heads_per_order;
+  pp.Dh = cfg->row_dim;
+  pp.E = pp.nh * cfg->row_dim;
+  pp.H = cfg->hidden;
+  pp.hc = cfg->hc_mult;
+  pp.dtype = cfg->dtype;
+  float* g = reinterpret_cast<float*>(w + L.g_off);
+  st = run_stage(cfg, pp, g, gates, s);
+  if (st != ENGRAM_OK) return st;
+  // u = g * V: the conv kernel without taps, one "sequence" of M positions
+  ConvParams cp;
+  memset(&cp, 0, sizeof cp);
+  cp.V = pp.V;
+  cp.g = g;
+  cp.conv_w = nullptr;
+  cp.Y = u;
+  cp.B = 1;
+  cp.T = static_cast<int32_t>(M);
+  if (M > INT32_MAX) return fail(ENGRAM_ERR_UNSUPPORTED, "M too large");
+  cp.H = cfg->hidden;
+  cp.hc = cfg->hc_mult;
+  cp.K = cfg->conv_kernel;
+  cp.dil = cfg->dilation;
+  cp.dtype = cfg->dtype;
+  return cuda_check(launch_gated_conv(cp, s), "gated value");
+}
+
+engram_status engram_short_conv(const engram_config* cfg, const void* u, int32_t B, int32_t T,
+                                const void* conv_w, void* conv_state, void* y,
+                                engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
+  if (static_cast<int64_t>(B) * T > 0 && (u == nullptr || y == nullptr || conv_w == nullptr))
+    return fail(ENGRAM_ERR_INVALID_ARG, "u / conv_w / y must be non-NULL");
+  if (u != nullptr && u == y) return fail(ENGRAM_ERR_INVALID_ARG, "u and y must not overlap");
+  ShortConvParams sp;
+  sp.u = u;
+  sp.conv_w = conv_w;
+  sp.state = conv_state;
+  sp.y = y;
+  sp.B = B;
+  sp.T = T;
+  sp.C = cfg->hc_mult * cfg->hidden;
+  sp.K = cfg->conv_kernel;
+  sp.dil = cfg->dilation;
+  sp.dtype = cfg->dtype;
+  return cuda_check(launch_short_conv(sp, static_cast<cudaStream_t>(stream)), "short conv");
+}
+
+engram_status engram_forward_workspace_size(const engram_config* cfg, int32_t B, int32_t T,
+                                            size_t* bytes) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (B < 0 || T < 0 || bytes == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "bad B/T/bytes");
+  *bytes = forward_layout(cfg, static_cast<int64_t>(B) * T).st.end;
+  return ENGRAM_OK;
+}
+
+engram_status engram_state_init(const engram_config* cfg, const engram_state* state, int32_t B,
+                                engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (state == nullptr || B < 0) return fail(ENGRAM_ERR_INVALID_ARG, "state NULL or B < 0");
+  const int n_hist = max_order(*cfg) - 1;
+  if (state->ring_len < (cfg->conv_kernel - 1) * cfg->dilation + 1)
+    return fail(ENGRAM_ERR_INVALID_ARG, "ring_len=%d < (K-1)*dilation+1", state->ring_len);
+  if ((n_hist > 0 && state->id_ring == nullptr) || state->v_ring == nullptr ||
+      state->g_ring == nullptr || state->pos == nullptr)
+    return fail(ENGRAM_ERR_INVALID_ARG, "a state array is NULL");
+  return cuda_check(launch_state_init(state->id_ring, n_hist, state->v_ring, state->g_ring,
+                                      state->pos, state->ring_len, B, cfg->hidden, cfg->hc_mult,
+                                      cfg->pad_id, cfg->dtype, static_cast<cudaStream_t>(stream)),
+                    "state init");
+}
+
+engram_status engram_forward(const engram_config* cfg, const engram_weights* wts,
+                             const int64_t* ids, int32_t B, int32_t T, const void* hidden,
+                             void* y, const engram_state* state, void* ws, size_t ws_bytes,
+                             uint32_t* dev_status, engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  st = check_dense_shapes(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (wts == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights is NULL");
+  if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
+  const int64_t M = static_cast<int64_t>(B) * T;
+  if (M == 0) return ENGRAM_OK;
+  const void* ptrs[] = {wts->table, wts->w_value, wts->w_key, wts->norm_key, wts->norm_query,
+                        wts->conv_w, hidden, y, ws, ids};
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "a tensor / workspace pointer is NULL");
+    if (!aligned16(p)) return fail(ENGRAM_ERR_INVALID_ARG, "tensor / workspace pointers must be 16-byte aligned");
+  }
+  if (wts->row_offsets == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "row_offsets (host) is NULL");
+  if (wts->lookup != nullptr && wts->raw_vocab < 1) return fail(ENGRAM_ERR_INVALID_ARG, "raw_vocab < 1");
+  if (wts->total_rows < 1 || wts->total_rows > INT32_MAX)
+    return fail(ENGRAM_ERR_UNSUPPORTED, "total_rows must be in [1, 2^31)");
+  HashParams hp;
+  st = fill_hash_params(cfg, wts->multipliers, wts->primes, &hp);
+  if (st != ENGRAM_OK) return st;
+  for (int h = 0; h < hp.nh; ++h) {
+    const int64_t off = wts->row_offsets[h];
+    if (off < 0 || off + wts->primes[h] > wts->total_rows)
+      return fail(ENGRAM_ERR_INVALID_ARG, "table %d (rows [%lld, %lld)) exceeds total_rows", h,
+                  static_cast<long long>(off), static_cast<long long>(off + wts->primes[h]));
+    hp.row_off[h] = off;
+  }
+  if (state != nullptr) {
+    if (state->ring_len < (cfg->conv_kernel - 1) * cfg->dilation + 1)
+      return fail(ENGRAM_ERR_INVALID_ARG, "state ring_len=%d < (K-1)*dilation+1", state->ring_len);
+    if ((hp.n_hist > 0 && state->id_ring == nullptr) || state->v_ring == nullptr ||
+        state->g_ring == nullptr || state->pos == nullptr)
+      return fail(ENGRAM_ERR_INVALID_ARG, "a state array is NULL");
+  }
+  const ForwardLayout L = forward_layout(cfg, M);
+  if (ws_bytes < L.st.end)
+    return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", ws_bytes, L.st.end);
+  char* w = static_cast<char*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // a1-a3: ids -> absolute table rows (head-major)
+  const int64_t ld = rows_ld(M);
+  int32_t* rows = reinterpret_cast<int32_t*>(w + L.rows_off);
+  hp.ids = ids;
+  hp.lookup = wts->lookup;
+  hp.raw_vocab = wts->raw_vocab;
+  hp.history = state != nullptr ? state->id_ring : nullptr;
+  hp.id_ring_out = state != nullptr ? state->id_ring : nullptr;
+  hp.rows_out = rows;
+  hp.ld_rows = ld;
+  hp.status = dev_status;
+  hp.B = B;
+  hp.T = T;
+  st = cuda_check(launch_hash(hp, s), "hash");
+  if (st != ENGRAM_OK) return st;
+
+  // a4-a7: gathered projection, score partials, gates
+  ProjParams pp;
+  memset(&pp, 0, sizeof pp);
+  pp.a_src = wts->table;
+  pp.rows = rows;
+  pp.ld_rows = ld;
+  pp.a_rows = wts->total_rows;
+  pp.w_value = wts->w_value;
+  pp.w_key = wts->w_key;
+  pp.norm_key = wts->norm_key;
+  pp.norm_query = wts->norm_query;
+  pp.hidden = hidden;
+  pp.V = w + L.st.v_off;
+  pp.partials = reinterpret_cast<float4*>(w + L.st.part_off);
+  pp.status = dev_status;
+  pp.M = M;
+  pp.nh = hp.nh;
+  pp.Dh = cfg->row_dim;
+  pp.E = hp.nh * cfg->row_dim;
+  pp.H = cfg->hidden;
+  pp.hc = cfg->hc_mult;
+  pp.dtype = cfg->dtype;
+  float* g = reinterpret_cast<float*>(w + L.st.g_off);
+  st = run_stage(cfg, pp, g, nullptr, s);
+  if (st != ENGRAM_OK) return st;
+
+  // a8-a9: gated value, short conv, residual
+  ConvParams cp;
+  memset(&cp, 0, sizeof cp);
+  cp.V = pp.V;
+  cp.g = g;
+  cp.conv_w = wts->conv_w;
+  cp.Y = y;
+  if (state != nullptr) {
+    cp.v_ring = state->v_ring;
+    cp.g_ring = state->g_ring;
+    cp.pos = state->pos;
+    cp.ring_len = state->ring_len;
+  }
+  cp.B = B;
+  cp.T = T;
+  cp.H = cfg->hidden;
+  cp.hc = cfg->hc_mult;
+  cp.K = cfg->conv_kernel;
+  cp.dil = cfg->dilation;
+  cp.dtype = cfg->dtype;
+  st = cuda_check(launch_gated_conv(cp, s), "gated conv");
+  if (st != ENGRAM_OK || state == nullptr) return st;
+
+  StateAdvanceParams ap;
+  ap.V = pp.V;
+  ap.g = g;
+  ap.v_ring = state->v_ring;
+  ap.g_ring = state->g_ring;
+  ap.pos = state->pos;
+  ap.ring_len = state->ring_len;
+  ap.B = B;
+  ap.T = T;
+  ap.H = cfg->hidden;
+  ap.hc = cfg->hc_mult;
+  ap.dtype = cfg->dtype;
+  return cuda_check(launch_state_advance(ap, s), "state advance");
+}
+
+}  // extern "C"

@@ -1,0 +1,197 @@
+// Internal interfaces of libengram: parameter blocks passed by value to the
+// kernels, the launchers each .cu file exports to the C-ABI layer, and small
+// device helpers shared by the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/engram.h"
+
+namespace engram {
+
+// ---------------------------------------------------------------- host side
+
+// Per-call parameters of the hash kernel (a1-a3).  The small per-head arrays
+// travel in the kernel's parameter space, so every thread reads them from the
+// constant bank.
+struct HashParams {
+  const int64_t* ids;       // [B, T] raw (lookup != null) or compressed ids
+  const int64_t* lookup;    // [raw_vocab] or null
+  const int64_t* history;   // [B, n_hist] or null (then pad_id)
+  int64_t* idx_out;         // [B*T, nh] int64 or null
+  int32_t* rows_out;        // [nh, ld_rows] absolute table rows (int32) or null
+  int64_t* id_ring_out;     // decode: [B, n_hist] ring written after use, or null
+  uint32_t* status;
+  int64_t raw_vocab;
+  int64_t vocab;
+  int64_t pad_id;
+  int64_t ld_rows;
+  int32_t B, T;
+  int32_t n_orders, J, nh, n_hist;
+  int32_t orders[ENGRAM_MAX_ORDERS];
+  uint64_t mult[ENGRAM_MAX_NGRAM];
+  uint64_t prime[ENGRAM_MAX_HEADS];
+  uint64_t barrett[ENGRAM_MAX_HEADS];   // floor((2^64 - 1) / p)
+  int64_t row_off[ENGRAM_MAX_HEADS];
+};
+cudaError_t launch_hash(const HashParams& p, cudaStream_t s);
+cudaError_t launch_compress(const int64_t* raw, int64_t n, const int64_t* lookup,
+                            int64_t raw_vocab, int64_t* out, uint32_t* status, cudaStream_t s);
+
+// Row gather (a4): e[m, h*Dh + c] = table[off[h] + idx[m, h], c].
+struct GatherParams {
+  const void* table;
+  const int64_t* idx;       // [M, nh]
+  void* e;                  // [M, nh*Dh]
+  uint32_t* status;
+  int64_t M;
+  int64_t total_rows;
+  int32_t nh;
+  int32_t row_bytes;
+  int64_t row_off[ENGRAM_MAX_HEADS];
+};
+cudaError_t launch_gather(const GatherParams& p, cudaStream_t s);
+
+// Projections (a5) with the per-tile score partial sums (a6) in the epilogue.
+// A is either gathered (rows != null: A[m, h*Dh..] = table[rows[h*ld_rows + m]])
+// or dense (rows == null: A = e [M, E]).  Outputs V [M, H] in dtype and
+// partials [M, hc, n_tiles] float4 = (sum K*nk*nq*Q, sum K^2, sum Q^2, 0)
+// over the tile's columns of branch h.
+struct ProjParams {
+  const void* a_src;        // table [*, Dh] (gathered) or e [M, E] (dense)
+  const int32_t* rows;      // [nh, ld_rows] or null
+  int64_t ld_rows;
+  int64_t a_rows;           // rows addressable in a_src (bounds of the TMA map)
+  const void* w_value;      // [H, E]
+  const void* w_key;        // [hc, H, E]
+  const void* norm_key;     // [hc, H]
+  const void* norm_query;   // [hc, H]
+  const void* hidden;       // [M, hc, H]
+  void* V;                  // [M, H]
+  float4* partials;         // [M, hc, n_tiles]
+  uint32_t* status;
+  int64_t M;
+  int32_t nh, Dh, E, H, hc;
+  int32_t n_tiles;          // column tiles per branch (H / tile width)
+  engram_dtype dtype;
+  uint32_t debug;
+};
+// Column-tile widths of the two projection engines (partials granularity).
+constexpr int kSimtTileN = 64;
+constexpr int kTcTileN = 256;
+bool tc_projection_supported(int Dh, int H, engram_dtype dt);
+cudaError_t launch_proj_simt(const ProjParams& p, cudaStream_t s);
+cudaError_t launch_proj_tc(const ProjParams& p, cudaStream_t s);
+
+// Gate finalisation (a6 reduction + a7): g[m, h] from the partials.
+struct GateParams {
+  const float4* partials;   // [M, hc, n_tiles]
+  float* g;                 // [M, hc]
+  float* g_copy;            // optional second output (API gates) or null
+  int64_t M;
+  int32_t hc, n_tiles, H;
+  float rms_eps, gate_eps;
+};
+cudaError_t launch_gate(const GateParams& p, cudaStream_t s);
+
+// Gated value + short conv + residual (a8, a9) from V and g.
+//   Y[b,t,h,c] = U(t) + sum_i w[h*H+c, i] U(t - (K-1-i) dil),  U(t) = g[t,h] V[t,c]
+// Positions before the chunk come from the state rings (if any) or are zero.
+// conv_w == null: Y = U (no conv; used by engram_gate_fuse).
+struct ConvParams {
+  const void* V;            // [B*T, H]
+  const float* g;           // [B*T, hc]
+  const void* conv_w;       // [hc*H, K] or null
+  void* Y;                  // [B*T, hc, H]
+  const void* v_ring;       // [B, ring_len, H] or null
+  const float* g_ring;      // [B, ring_len, hc]
+  const int64_t* pos;       // [B]
+  int32_t ring_len;
+  int32_t B, T, H, hc, K, dil;
+  engram_dtype dtype;
+};
+cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s);
+
+// Standalone short conv over a materialised u (engram_short_conv).
+struct ShortConvParams {
+  const void* u;            // [B, T, C]
+  const void* conv_w;       // [C, K]
+  void* state;              // [B, (K-1)*dil, C] or null
+  void* y;                  // [B, T, C]
+  int32_t B, T, C, K, dil;
+  engram_dtype dtype;
+};
+cudaError_t launch_short_conv(const ShortConvParams& p, cudaStream_t s);
+
+// Streaming state: write this chunk's last V/g rows into the rings, advance pos.
+struct StateAdvanceParams {
+  const void* V;            // [B*T, H]
+  const float* g;           // [B*T, hc]
+  void* v_ring;
+  float* g_ring;
+  int64_t* pos;
+  int32_t ring_len;
+  int32_t B, T, H, hc;
+  engram_dtype dtype;
+};
+cudaError_t launch_state_advance(const StateAdvanceParams& p, cudaStream_t s);
+cudaError_t launch_state_init(int64_t* id_ring, int n_hist, void* v_ring, float* g_ring,
+                              int64_t* pos, int32_t ring_len, int32_t B, int32_t H, int32_t hc,
+                              int64_t pad_id, engram_dtype dt, cudaStream_t s);
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// ---------------------------------------------------------------- device side
+
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
+  if (status != nullptr) atomicOr(status, bits);
+}
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t v) {
+  return __uint_as_float(static_cast<uint32_t>(v) << 16);
+}
+
+// Round-to-nearest-even float -> bfloat16 (the cuda_bf16 intrinsic).
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float load(const float* p, int64_t i) { return __ldg(p + i); }
+  static __device__ __forceinline__ void store(float* p, int64_t i, float v) { p[i] = v; }
+};
+template <> struct Elem<uint16_t> {
+  static __device__ __forceinline__ float load(const uint16_t* p, int64_t i) {
+    return bf16_to_f32(__ldg(p + i));
+  }
+  static __device__ __forceinline__ void store(uint16_t* p, int64_t i, float v) {
+    p[i] = f32_to_bf16(v);
+  }
+};
+
+// Exact x mod p for x < 2^64, p >= 2, with mu = floor((2^64 - 1) / p)
+// (Barrett reduction: the estimate q = floor(x * mu / 2^64) is at most one
+// below floor(x / p), so one conditional subtraction suffices; a second is
+// kept for safety).
+__device__ __forceinline__ uint64_t barrett_mod(uint64_t x, uint64_t p, uint64_t mu) {
+  uint64_t q = __umul64hi(x, mu);
+  uint64_t r = x - q * p;
+  if (r >= p) r -= p;
+  if (r >= p) r -= p;
+  return r;
+}
+
+// Gate of formulas §2.2 step 2: sigmoid(sign(s) * sqrt(max(|s|, eps))), sign(0) = 0.
+__device__ __forceinline__ float gate_from_score(float s, float gate_eps) {
+  float a = fmaxf(fabsf(s), gate_eps);
+  float sg = (s > 0.f) ? 1.f : ((s < 0.f) ? -1.f : 0.f);
+  float z = sqrtf(a) * sg;
+  return 1.f / (1.f + expf(-z));
+}
+
+}  // namespace engram

@@ -1,0 +1,158 @@
+// K1: compressed-id lookup + time shift + multi-head n-gram hash, one pass.
+//
+//   x       = lookup[raw]                                   explainer §2.2 1), §4.1
+//   tok_k   = x[t-k], pad_id (or the history) for t-k < 0   formulas §4.2-4.3
+//   mix_o   = xor_{k < n_o} tok_k * m_k   (int64)           formulas §1.2 step 1
+//   idx_o,j = mix_o mod p_o,j                               formulas §1.2 step 2, §1.3
+//
+// Layout of the work: one warp owns 32 consecutive positions of one sequence.
+// Lane l loads x[t0 + l]; lanes l < n_hist also load the n_hist ids before t0
+// (or pad / history), so every n-gram window is assembled with warp shuffles
+// instead of re-reading memory.  Each lane then computes the mix of every
+// order for its position (64-bit integer multiply and xor) and reduces it by
+// each head's prime with an exact Barrett reduction (the GPU has no 64-bit
+// divide).  Outputs are either the API's idx [M, nh] (int64) or, inside
+// engram_forward, absolute int32 table rows laid out head-major [nh, M] so the
+// projection's row gather reads 128 consecutive rows of one head with one
+// coalesced load.
+#include "engram_internal.cuh"
+
+namespace engram {
+
+namespace {
+
+__device__ __forceinline__ int64_t load_id(const HashParams& p, int64_t raw) {
+  int64_t x = raw;
+  if (p.lookup != nullptr) {
+    if (raw < 0 || raw >= p.raw_vocab) {
+      set_status(p.status, ENGRAM_STATUS_ID_RANGE);
+      return p.pad_id;
+    }
+    x = __ldg(p.lookup + raw);
+  }
+  if (x < 0 || x >= p.vocab) {
+    set_status(p.status, ENGRAM_STATUS_ID_RANGE);
+    return p.pad_id;
+  }
+  return x;
+}
+
+__global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashParams p) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int b = blockIdx.y;
+  const int t0 = blockIdx.x * 256 + warp * 32;
+  if (t0 >= p.T) return;  // whole warp past the end (warp-uniform)
+  const int t = t0 + lane;
+  const int64_t base = static_cast<int64_t>(b) * p.T;
+
+  // the id at this lane's position
+  int64_t x = p.pad_id;
+  if (t < p.T) x = load_id(p, __ldg(p.ids + base + t));
+
+  // the n_hist ids before t0 (lane l holds position t0 - n_hist + l)
+  int64_t halo = p.pad_id;
+  if (lane < p.n_hist) {
+    int th = t0 - p.n_hist + lane;
+    if (th >= 0) {
+      halo = load_id(p, __ldg(p.ids + base + th));
+    } else if (p.history != nullptr) {
+      // history: previous ids of this sequence, most recent last (already compressed)
+      int64_t hv = __ldg(p.history + static_cast<int64_t>(b) * p.n_hist + p.n_hist + th);
+      if (hv < 0 || hv >= p.vocab) {
+        set_status(p.status, ENGRAM_STATUS_ID_RANGE);
+        hv = p.pad_id;
+      }
+      halo = hv;
+    }
+  }
+
+  // tok[k] = id at position t - k, assembled by shuffles (warp-cooperative padding)
+  uint64_t tok[ENGRAM_MAX_NGRAM];
+#pragma unroll
+  for (int k = 0; k < ENGRAM_MAX_NGRAM; ++k) {
+    int64_t from_x = __shfl_sync(0xffffffffu, x, (lane - k) & 31);
+    int64_t from_h = __shfl_sync(0xffffffffu, halo, (p.n_hist + lane - k) & 31);
+    tok[k] = static_cast<uint64_t>(lane >= k ? from_x : from_h);
+  }
+
+  if (t >= p.T) return;
+  const int64_t m = base + t;
+#pragma unroll 1
+  for (int o = 0; o < p.n_orders; ++o) {
+    const int n = p.orders[o];
+    uint64_t mix = tok[0] * p.mult[0];
+#pragma unroll
+    for (int k = 1; k < ENGRAM_MAX_NGRAM; ++k)
+      if (k < n) mix ^= tok[k] * p.mult[k];
+#pragma unroll 1
+    for (int j = 0; j < p.J; ++j) {
+      const int h = o * p.J + j;
+      const uint64_t r = barrett_mod(mix, p.prime[h], p.barrett[h]);
+      if (p.idx_out != nullptr) p.idx_out[m * p.nh + h] = static_cast<int64_t>(r);
+      if (p.rows_out != nullptr)
+        p.rows_out[static_cast<int64_t>(h) * p.ld_rows + m] = static_cast<int32_t>(p.row_off[h] + static_cast<int64_t>(r));
+    }
+  }
+}
+
+// Decode / chunked prefill: after the hash of this chunk has read the old ring,
+// the ring becomes the last n_hist ids of (old ring ++ chunk).  One thread per
+// sequence; it runs after hash_kernel on the same stream.
+__global__ void id_ring_kernel(const __grid_constant__ HashParams p) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= p.B) return;
+  int64_t* ring = p.id_ring_out + static_cast<int64_t>(b) * p.n_hist;
+  const int64_t base = static_cast<int64_t>(b) * p.T;
+  // ascending j reads index j + T >= j before writing j (in-place forward shift)
+  for (int j = 0; j < p.n_hist; ++j) {
+    int src = j + p.T;  // position in (old ring ++ chunk)
+    int64_t v;
+    if (src < p.n_hist) v = ring[src];
+    else v = load_id(p, __ldg(p.ids + base + (src - p.n_hist)));
+    ring[j] = v;
+  }
+}
+
+__global__ void compress_kernel(const int64_t* __restrict__ raw, int64_t n,
+                                const int64_t* __restrict__ lookup, int64_t raw_vocab,
+                                int64_t* __restrict__ out, uint32_t* status) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int64_t r = __ldg(raw + i);
+    if (r < 0 || r >= raw_vocab) {
+      set_status(status, ENGRAM_STATUS_ID_RANGE);
+      out[i] = -1;
+    } else {
+      out[i] = __ldg(lookup + r);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_hash(const HashParams& p, cudaStream_t s) {
+  if (p.B > 0 && p.T > 0) {
+    dim3 grid((p.T + 255) / 256, p.B);
+    hash_kernel<<<grid, 256, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (p.id_ring_out != nullptr && p.n_hist > 0 && p.B > 0) {
+    id_ring_kernel<<<(p.B + 127) / 128, 128, 0, s>>>(p);
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_compress(const int64_t* raw, int64_t n, const int64_t* lookup,
+                            int64_t raw_vocab, int64_t* out, uint32_t* status, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  int cap = num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  compress_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(raw, n, lookup, raw_vocab, out, status);
+  return cudaGetLastError();
+}
+
+}  // namespace engram

@@ -1,0 +1,233 @@
+/*
+ * libengram: the Engram conditional-memory forward pass on NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page and section throughout:
+ *   formulas page  = the Engram formula document at kwkr.cn/news/37585
+ *   explainer page = the Engram paper walk-through at yaoyuxiang.cn/news/830577
+ *   (the extracted pages print no titles; they are named by their subject)
+ *
+ * The pass (explainer §4.3 forward walk-through; formulas §5.2 data flow):
+ *   ids --(lookup)--> compressed ids x                      explainer §2.2 1), §4.1
+ *   tokens[k] = shift_k(x), pad_id before the start         formulas §4.2-4.3
+ *   idx[o,j] = (xor_k tokens[k]*m_k) mod p[o,j]             formulas §1.2-1.3; explainer §4.2
+ *   e = concat_{o,j} Table[o,j][idx[o,j]]                   explainer §2.2 1), §4.3
+ *   V = e Wv^T;  K_h = e Wk_h^T  (h < hc_mult)              formulas §2.2 steps 1, 3; explainer §2.2 4)
+ *   s_h = sum(RMSNorm(K_h; nk_h) * RMSNorm(Q_h; nq_h)) / sqrt(H),  Q_h = hidden[..., h, :]
+ *                                                           formulas §2.2 step 1
+ *   g_h = sigmoid(sign(s_h) * sqrt(max(|s_h|, gate_eps)))   formulas §2.2 step 2
+ *   U_h = g_h * V;  Y_h = U_h + depthwise causal conv(U_h)  formulas §2.2 step 3, §3.2;
+ *         (kernel K, dilation = max n-gram order)           explainer §2.2 3)
+ *
+ * Conventions for every entry point:
+ *  - Tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *    row-major, in the layouts stated per argument.  Arrays marked HOST are
+ *    read on the host during the call and may be freed when it returns.
+ *  - The library never allocates device memory; scratch space is passed in
+ *    (see the *_workspace_size queries).  It never synchronises the device or
+ *    the stream, except engram_read_status which says so.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and returns an engram_status for host-side argument
+ *    checks and launch errors.  Conditions found on the device (ids out of
+ *    range, a pipeline wait that ran out) are OR-ed into *dev_status (a device
+ *    uint32_t, may be NULL) as ENGRAM_STATUS_* bits; read them with
+ *    engram_read_status after the work completes.
+ *  - Floating tensors are all of the config's dtype (float32 or bfloat16);
+ *    all accumulation is float32.
+ *  - On a non-OK return nothing was launched; engram_last_error gives text.
+ */
+#ifndef ENGRAM_H
+#define ENGRAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ENGRAM_MAX_ORDERS 8   /* distinct n-gram orders */
+#define ENGRAM_MAX_NGRAM 8    /* largest n-gram order */
+#define ENGRAM_MAX_HEADS 64   /* orders x heads per order */
+#define ENGRAM_MAX_HC 8       /* hyper-connection branches */
+#define ENGRAM_MAX_CONV_K 8   /* short-conv kernel length */
+
+typedef enum {
+  ENGRAM_OK = 0,
+  ENGRAM_ERR_INVALID_ARG = 1, /* null pointer, bad size, range, alignment */
+  ENGRAM_ERR_UNSUPPORTED = 2, /* valid but not supported by this build (dtype/shape) */
+  ENGRAM_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  ENGRAM_ERR_TIMEOUT = 4,     /* device reported ENGRAM_STATUS_TIMEOUT */
+  ENGRAM_ERR_ID_RANGE = 5     /* device reported ENGRAM_STATUS_ID_RANGE / _ROW_RANGE */
+} engram_status;
+
+typedef enum { ENGRAM_F32 = 0, ENGRAM_BF16 = 1 } engram_dtype;
+
+/* A cudaStream_t, passed as a plain pointer so this header needs no CUDA headers. */
+typedef void* engram_stream;
+
+/* Bits a kernel may OR into *dev_status. */
+#define ENGRAM_STATUS_ID_RANGE 0x1u  /* an id outside [0, vocab) (or a raw id outside the
+                                        lookup); it was replaced by pad_id */
+#define ENGRAM_STATUS_ROW_RANGE 0x2u /* a gathered row outside the table; zeros were written */
+#define ENGRAM_STATUS_TIMEOUT 0x4u   /* a bounded pipeline wait ran out; that call's outputs
+                                        are not valid (no hang, no trap: the kernel returned) */
+
+/* Shape of one Engram layer (explainer §4.3; formulas §1.2, §1.4, §2.2, §4.2). */
+typedef struct {
+  int32_t n_orders;                   /* number of n-gram orders, 1..ENGRAM_MAX_ORDERS */
+  int32_t orders[ENGRAM_MAX_ORDERS];  /* ascending n-gram sizes, 1..ENGRAM_MAX_NGRAM */
+  int32_t heads_per_order;            /* J: hash heads (one prime each) per order */
+  int32_t row_dim;                    /* Dh: width of one table row; E = n_orders*J*Dh */
+  int32_t hidden;                     /* H: backbone hidden size (d in sqrt(d)) */
+  int32_t hc_mult;                    /* hc: hyper-connection branches, 1..ENGRAM_MAX_HC */
+  int32_t conv_kernel;                /* K: short-conv taps (the pages use 4) */
+  int32_t dilation;                   /* conv dilation (the pages: the largest order) */
+  int64_t pad_id;                     /* id used before the sequence start, in [0, 2^32) */
+  int64_t vocab;                      /* compressed vocabulary size, 1..2^32 */
+  float rms_eps;                      /* RMSNorm epsilon (> 0; 1e-6 in the workloads) */
+  float gate_eps;                     /* floor of |s| under the square root (1e-6) */
+  engram_dtype dtype;                 /* storage type of every floating tensor */
+} engram_config;
+
+/* Parameters of one Engram layer. */
+typedef struct {
+  const void* table;           /* DEVICE [total_rows, Dh]: the per-(order, head) tables stacked
+                                  in (order asc, head asc) order (explainer §4.3) */
+  int64_t total_rows;          /* rows in `table` */
+  const int64_t* row_offsets;  /* HOST [nh]: first row of table (o, j) at index o*J + j */
+  const int64_t* primes;       /* HOST [nh]: modulus p[o,j], 2 <= p < 2^31 (formulas §1.2 step 2) */
+  const int64_t* multipliers;  /* HOST [max order]: odd m_k, 0 < m_k < 2^31 (formulas §1.2);
+                                  m_0 multiplies the current token */
+  const int64_t* lookup;       /* DEVICE [raw_vocab] raw -> compressed id, or NULL when the ids
+                                  are already compressed (explainer §2.2 1)) */
+  int64_t raw_vocab;           /* entries in `lookup` */
+  const void* w_value;         /* DEVICE [H, E]: value projection (shared by branches) */
+  const void* w_key;           /* DEVICE [hc, H, E]: one key projection per branch */
+  const void* norm_key;        /* DEVICE [hc, H]: RMSNorm weights of the keys */
+  const void* norm_query;      /* DEVICE [hc, H]: RMSNorm weights of the queries */
+  const void* conv_w;          /* DEVICE [hc*H, K]: depthwise conv taps, PyTorch Conv1d order
+                                  (tap K-1 multiplies the current position) */
+} engram_weights;
+
+/* Streaming state of B sequences for engram_forward (decode or chunked prefill).
+ * Initialise with engram_state_init; pass the same state to consecutive calls. */
+typedef struct {
+  int64_t* id_ring;  /* DEVICE [B, max_order-1]: last compressed ids, most recent last */
+  void* v_ring;      /* DEVICE [B, ring_len, H] (dtype): V of recent positions, slot = pos % ring_len */
+  float* g_ring;     /* DEVICE [B, ring_len, hc]: gates of recent positions */
+  int64_t* pos;      /* DEVICE [B]: tokens consumed so far per sequence */
+  int32_t ring_len;  /* >= (K-1)*dilation + 1 */
+} engram_state;
+
+/* ---- housekeeping ---------------------------------------------------- */
+
+/* Library version as 10000*major + 100*minor + patch. */
+int32_t engram_version(void);
+
+/* Copies the calling thread's last error message (NUL-terminated, truncated to n). */
+size_t engram_last_error(char* buf, size_t n);
+
+/* Synchronises `stream`, copies *dev_status to *host_bits and clears the device
+ * word.  Returns ENGRAM_ERR_TIMEOUT / ENGRAM_ERR_ID_RANGE if those bits are set. */
+engram_status engram_read_status(uint32_t* dev_status, uint32_t* host_bits, engram_stream stream);
+
+/* Test knobs (process-wide).  ENGRAM_DEBUG_FORCE_TIMEOUT makes the next
+ * projection launches wait, with a short limit, on a barrier nothing arrives
+ * at, so the timeout path runs without a hang.  ENGRAM_DEBUG_FORCE_SIMT selects
+ * the CUDA-core projection kernel even where the tensor-core one applies. */
+#define ENGRAM_DEBUG_FORCE_TIMEOUT 0x1u
+#define ENGRAM_DEBUG_FORCE_SIMT 0x2u
+void engram_set_debug(uint32_t flags);
+
+/* Which projection engine engram_forward / engram_gate_fuse use for cfg under
+ * the current debug flags: ENGRAM_ENGINE_TCGEN05 (tensor cores, bfloat16,
+ * Dh == 64, H % 256 == 0) or ENGRAM_ENGINE_SIMT (CUDA cores); -1 if cfg is
+ * invalid. */
+#define ENGRAM_ENGINE_SIMT 0
+#define ENGRAM_ENGINE_TCGEN05 1
+int32_t engram_projection_engine(const engram_config* cfg);
+
+/* ---- steps of the pass ----------------------------------------------- */
+
+/* a1. out[i] = lookup[raw[i]]  (explainer §2.2 1), §4.1: the normalised-tokenizer
+ * lookup).  raw, out: DEVICE int64 [n]; lookup: DEVICE int64 [raw_vocab].
+ * A raw id outside [0, raw_vocab) sets ENGRAM_STATUS_ID_RANGE and writes -1. */
+engram_status engram_compress_ids(const int64_t* raw, int64_t n, const int64_t* lookup,
+                                  int64_t raw_vocab, int64_t* out, uint32_t* dev_status,
+                                  engram_stream stream);
+
+/* a2+a3. N-gram hash (formulas §1.2 steps 1-2, §1.3, §4.2-4.3; explainer §4.2):
+ *   idx[b, t, o*J + j] = (xor_{k < n_o} x[b, t-k] * m_k) mod p[o*J + j]
+ * where x[b, t-k] for t-k < 0 is history[b, max_n-1 + t-k] when `history` is
+ * given (DEVICE int64 [B, max_n-1], most recent last) and pad_id otherwise.
+ * ids: DEVICE int64 [B, T] compressed ids; idx: DEVICE int64 [B, T, nh].
+ * multipliers: HOST [max order]; primes: HOST [nh].
+ * An id outside [0, vocab) sets ENGRAM_STATUS_ID_RANGE and hashes as pad_id. */
+engram_status engram_hash(const engram_config* cfg, const int64_t* ids, int32_t B, int32_t T,
+                          const int64_t* history, const int64_t* multipliers,
+                          const int64_t* primes, int64_t* idx, uint32_t* dev_status,
+                          engram_stream stream);
+
+/* a4. Row gather and concatenation (explainer §2.2 1), §4.3):
+ *   e[m, h*Dh + c] = table[row_offsets[h] + idx[m, h], c]   (a bit-exact copy)
+ * table: DEVICE [total_rows, Dh]; row_offsets: HOST [nh]; idx: DEVICE int64 [M, nh];
+ * e: DEVICE [M, nh*Dh].  A row outside [0, total_rows) sets
+ * ENGRAM_STATUS_ROW_RANGE and writes zeros for that row. */
+engram_status engram_gather(const engram_config* cfg, const void* table, int64_t total_rows,
+                            const int64_t* row_offsets, const int64_t* idx, int64_t M,
+                            void* e, uint32_t* dev_status, engram_stream stream);
+
+/* a5-a8. Projections, gate and gated value from gathered embeddings
+ * (formulas §2.2 steps 1-3; explainer §2.2 2) 4), §4.3):
+ *   u[m, h, :] = g[m, h] * (e[m] Wv^T),  g = gate of RMSNorm(e Wk_h^T) . RMSNorm(hidden[m, h])
+ * e: DEVICE [M, E]; hidden: DEVICE [M, hc, H]; u: DEVICE [M, hc, H];
+ * gates: DEVICE float [M, hc] or NULL.  ws: DEVICE scratch of
+ * engram_gate_fuse_workspace_size bytes, 256-byte aligned. */
+engram_status engram_gate_fuse_workspace_size(const engram_config* cfg, int64_t M, size_t* bytes);
+engram_status engram_gate_fuse(const engram_config* cfg, const void* e, const void* w_value,
+                               const void* w_key, const void* norm_key, const void* norm_query,
+                               const void* hidden, int64_t M, void* u, float* gates, void* ws,
+                               size_t ws_bytes, uint32_t* dev_status, engram_stream stream);
+
+/* a9. Short conv + residual (formulas §3.2; explainer §2.2 3)):
+ *   y[b, t, ch] = u[b, t, ch] + sum_{i<K} conv_w[ch, i] * u[b, t - (K-1-i)*dil, ch]
+ * over channels ch = h*H + c.  u, y: DEVICE [B, T, hc*H].  Positions before the
+ * start read conv_state when given (DEVICE [B, (K-1)*dil, hc*H], oldest first),
+ * else zero; when given, conv_state is updated in place to the last (K-1)*dil
+ * positions of (old state ++ u).  u and y must not overlap. */
+engram_status engram_short_conv(const engram_config* cfg, const void* u, int32_t B, int32_t T,
+                                const void* conv_w, void* conv_state, void* y,
+                                engram_stream stream);
+
+/* ---- the whole pass --------------------------------------------------- */
+
+/* Scratch bytes engram_forward needs for B sequences of T tokens. */
+engram_status engram_forward_workspace_size(const engram_config* cfg, int32_t B, int32_t T,
+                                            size_t* bytes);
+
+/* Fills a state for B sequences: ids = pad_id, rings and positions = 0. */
+engram_status engram_state_init(const engram_config* cfg, const engram_state* state, int32_t B,
+                                engram_stream stream);
+
+/* Engram.forward(hidden_states, input_ids) of the explainer page §4.3, all steps
+ * a1-a9 on the device.
+ *   ids:    DEVICE int64 [B, T]; raw ids when weights->lookup is set, else compressed
+ *   hidden: DEVICE [B, T, hc, H];  y: DEVICE [B, T, hc, H]
+ *   state:  NULL for an independent prefill; otherwise the sequences continue
+ *           from the state (positions before this call come from its rings) and
+ *           the state is advanced by T tokens.  256 calls with T = 1 produce the
+ *           same y as one prefill over T = 256.
+ *   ws:     DEVICE scratch of engram_forward_workspace_size(cfg, B, T) bytes,
+ *           256-byte aligned.
+ * Requirements: H % 64 == 0; bfloat16 with Dh == 64 and H % 256 == 0 runs the
+ * tensor-core (tcgen05) projection, other shapes the CUDA-core one. */
+engram_status engram_forward(const engram_config* cfg, const engram_weights* weights,
+                             const int64_t* ids, int32_t B, int32_t T, const void* hidden,
+                             void* y, const engram_state* state, void* ws, size_t ws_bytes,
+                             uint32_t* dev_status, engram_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENGRAM_H */

@@ -6,8 +6,9 @@
  * code, header, table or helper with the CUDA library and never calls it.
  *
  * Sources (cited by page and section):
- *   "formulas page"  = Engram 核心数学公式说明 (kwkr.cn/news/37585)
- *   "explainer page" = Engram 条件记忆解读 (yaoyuxiang.cn/news/830577)
+ *   "formulas page"  = the Engram formula document at kwkr.cn/news/37585
+ *   "explainer page" = the Engram paper walk-through at yaoyuxiang.cn/news/830577
+ *   (the extracted pages print no titles; they are named by their subject)
  *
  * Every step is written out as its definition, in the pages' order, with no
  * blocking or reordering:

@@ -1,0 +1,106 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function
+include/engram.h declares, and rejects bad arguments on the host before any
+launch (no compute calls here)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+import torch
+
+from hashed_gram_conditional_hash_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "engram.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(engram_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 13
+    lib = C.CDLL(L.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_error_text():
+    assert L.engram_version() >= 100
+    cfg = L.make_config((2, 3), 4, 32, 256, 1, 4, 3, 0, 1580, torch.float32)
+    cfg.n_orders = 0
+    n = C.c_size_t(0)
+    assert L.lib().engram_forward_workspace_size(C.byref(cfg), 1, 8, C.byref(n)) == 1
+    assert "n_orders" in L.last_error()
+
+
+def _cfg(**kw):
+    c = L.make_config((2, 3), 2, 64, 256, 2, 4, 3, 0, 5000, torch.bfloat16)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("field,value", [
+    ("heads_per_order", 0), ("heads_per_order", 40), ("hc_mult", 9), ("conv_kernel", 0),
+    ("dilation", 0), ("pad_id", -1), ("pad_id", 1 << 32), ("vocab", 0), ("rms_eps", 0.0),
+    ("dtype", 7)])
+def test_config_validation(field, value):
+    n = C.c_size_t(0)
+    cfg = _cfg(**{field: value})
+    assert L.lib().engram_forward_workspace_size(C.byref(cfg), 2, 8, C.byref(n)) == 1
+
+
+def test_orders_must_ascend():
+    cfg = _cfg()
+    cfg.orders[1] = 2
+    n = C.c_size_t(0)
+    assert L.lib().engram_forward_workspace_size(C.byref(cfg), 2, 8, C.byref(n)) == 1
+
+
+@pytest.mark.parametrize("mult,primes", [
+    ([2, 3, 5], [101] * 4),               # even multiplier
+    ([1 << 31, 3, 5], [101] * 4),         # multiplier too large
+    ([1, 3, 5], [1, 101, 103, 107]),      # modulus < 2
+    ([1, 3, 5], [1 << 31, 101, 103, 107]),
+])
+def test_hash_parameter_validation(mult, primes):
+    cfg = _cfg()
+    m = (C.c_int64 * 3)(*mult)
+    p = (C.c_int64 * 4)(*primes)
+    # pointers are never dereferenced: the call fails on the host first
+    rc = L.lib().engram_hash(C.byref(cfg), C.c_void_p(16), 1, 4, None, m, p, C.c_void_p(16),
+                             None, None)
+    assert rc == 1
+
+
+def test_workspace_sizes_grow_with_tokens():
+    cfg = _cfg()
+    a = L.engram_forward_workspace_size(cfg, 1, 128)
+    b = L.engram_forward_workspace_size(cfg, 4, 128)
+    assert 0 < a < b and a % 256 == 0 and b % 256 == 0
+    assert L.engram_gate_fuse_workspace_size(cfg, 512) > 0
+
+
+def test_forward_rejects_null_and_misaligned():
+    cfg = _cfg()
+    w = L.EngramWeights()
+    ws_n = L.engram_forward_workspace_size(cfg, 1, 4)
+    rc = L.lib().engram_forward(C.byref(cfg), C.byref(w), C.c_void_p(256), 1, 4, C.c_void_p(256),
+                                C.c_void_p(256), None, C.c_void_p(256), ws_n, None, None)
+    assert rc == 1 and "NULL" in L.last_error()
+    for f in ("table", "w_value", "w_key", "norm_key", "norm_query", "conv_w"):
+        setattr(w, f, 4096)
+    w.table = 4100  # not 16-byte aligned
+    rc = L.lib().engram_forward(C.byref(cfg), C.byref(w), C.c_void_p(256), 1, 4, C.c_void_p(256),
+                                C.c_void_p(256), None, C.c_void_p(256), ws_n, None, None)
+    assert rc == 1 and "aligned" in L.last_error()
+
+
+def test_short_conv_rejects_aliasing():
+    cfg = _cfg()
+    rc = L.lib().engram_short_conv(C.byref(cfg), C.c_void_p(256), 1, 4, C.c_void_p(512), None,
+                                   C.c_void_p(256), None)
+    assert rc == 1

@@ -1,0 +1,137 @@
+"""GPU parity of engram_forward (the whole pass through the C ABI) against the
+float64 oracle: full comparison on few-tile shapes with ragged tails, sampled
+positions (sequence edges + random interior) on the full-size workloads in
+the launch configuration the benchmark times, plus degenerate cases."""
+import numpy as np
+import pytest
+import torch
+
+from hashed_gram_conditional_hash_b200 import EngramLayer
+from hashed_gram_conditional_hash_b200 import _lib as L
+from hashed_gram_conditional_hash_b200 import workloads as W
+
+from gpu_helpers import (TOL, device_params, oracle_at, oracle_forward_full, rel_err,
+                         sample_positions)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run(p, engine="auto", conv_w=None):
+    if engine == "simt":
+        L.engram_set_debug(L.DEBUG_FORCE_SIMT)
+    try:
+        layer = EngramLayer.from_params(p)
+        if conv_w is not None:
+            layer.weights.conv_w = conv_w.data_ptr()
+        st = torch.zeros(1, dtype=torch.int32, device=DEV)
+        y = layer.forward(p.ids, p.hidden, dev_status=st)
+        assert L.engram_read_status(st) == 0
+        return y
+    finally:
+        L.engram_set_debug(0)
+
+
+SMALL = [
+    dict(),                                                        # bf16, B=3, T=77, hc=2
+    dict(B=2, T=130, hidden=512, hc_mult=4, orders=(2, 3, 4), dilation=4),
+    dict(B=1, T=1),
+    dict(B=4, T=3, hc_mult=1),
+    dict(dtype="f32", B=2, T=50, row_dim=32, hidden=128, hc_mult=3),
+    dict(B=2, T=200, heads_per_order=4, hidden=768, hc_mult=2),   # 768 = 3 tiles of 256
+]
+
+
+@pytest.mark.parametrize("kw", SMALL, ids=[str(i) for i in range(len(SMALL))])
+@pytest.mark.parametrize("engine", ["auto", "simt"])
+def test_forward_small_full(kw, engine):
+    w = W.small_workload(**kw)
+    p = device_params(w)
+    y = _run(p, engine)
+    ref = oracle_forward_full(p)
+    assert rel_err(y.double().cpu().numpy(), ref["Y"]) <= TOL[w.dtype]
+
+
+def test_forward_tiny_f32_full():
+    w = W.CONFIGS["tiny_f32"]
+    p = device_params(w)
+    y = _run(p)
+    ref = oracle_forward_full(p)
+    err = rel_err(y.double().cpu().numpy(), ref["Y"])
+    assert err <= TOL["f32"], err
+
+
+@pytest.mark.parametrize("name,n_random", [("model_bf16", 48), ("large_table_bf16", 24),
+                                           ("hbm_table_bf16", 16)])
+def test_forward_full_size_sampled(name, n_random):
+    w = W.CONFIGS[name]
+    p = device_params(w)
+    y = _run(p)
+    pos = sample_positions(w.B, w.T, w.dil, n_random, seed=11)
+    Yref, s, g, _ = oracle_at(p, pos)
+    got = torch.stack([y[b, t] for b, t in pos]).double().cpu().numpy()
+    err = rel_err(got, Yref)
+    assert err <= TOL[w.dtype], err
+
+
+def test_forward_zero_conv_is_gated_value():
+    w = W.small_workload(B=2, T=40)
+    p = device_params(w)
+    zero = torch.zeros_like(p.conv_w)
+    y = _run(p, conv_w=zero)
+    ref = oracle_forward_full(p, conv_w=zero)
+    assert rel_err(y.double().cpu().numpy(), ref["g"][..., None] * ref["V"][:, :, None, :]) <= TOL["bf16"]
+
+
+def test_forward_engines_agree():
+    w = W.small_workload(B=2, T=300, hidden=512, hc_mult=4)
+    p = device_params(w)
+    a = _run(p, "auto").double()
+    b = _run(p, "simt").double()
+    assert (a - b).abs().max().item() <= 2e-2 * b.abs().max().item()
+
+
+def test_forward_empty_is_noop():
+    w = W.small_workload()
+    p = device_params(w)
+    layer = EngramLayer.from_params(p)
+    ids = torch.empty((0, 5), dtype=torch.int64, device=DEV)
+    hid = torch.empty((0, 5, w.hc_mult, w.hidden), dtype=w.torch_dtype, device=DEV)
+    y = layer.forward(ids, hid)
+    assert y.shape == (0, 5, w.hc_mult, w.hidden)
+
+
+def test_forward_flags_out_of_range_ids():
+    w = W.small_workload(B=1, T=16)
+    p = device_params(w)
+    p.ids[0, 3] = w.vocab + 10
+    layer = EngramLayer.from_params(p)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    layer.forward(p.ids, p.hidden, dev_status=st)
+    assert L.engram_read_status(st) & L.STATUS_ID_RANGE
+
+
+def test_forward_timeout_path_returns_and_context_survives():
+    w = W.small_workload(B=2, T=64)
+    p = device_params(w)
+    layer = EngramLayer.from_params(p)
+    if not _tc_active(w):
+        pytest.skip("tensor-core engine not active for this shape")
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    L.engram_set_debug(L.DEBUG_FORCE_TIMEOUT)
+    try:
+        layer.forward(p.ids, p.hidden, dev_status=st)
+        bits = L.engram_read_status(st)
+    finally:
+        L.engram_set_debug(0)
+    assert bits & L.STATUS_TIMEOUT
+    # the context is still usable and the next call is correct
+    y = _run(p)
+    ref = oracle_forward_full(p)
+    assert rel_err(y.double().cpu().numpy(), ref["Y"]) <= TOL["bf16"]
+
+
+def _tc_active(w) -> bool:
+    cfg = L.make_config(w.orders, w.heads_per_order, w.row_dim, w.hidden, w.hc_mult,
+                        w.conv_kernel, w.dil, w.pad_id, w.vocab, w.torch_dtype)
+    return L.engram_projection_engine(cfg) == L.ENGINE_TCGEN05
