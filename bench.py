@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Engram forward benchmark: tokens/s of engram_forward on B200.
+
+One step = one engram_forward over one batch of the workload (hash -> gathered
+tcgen05 projection + score partials -> gate -> gated value + short conv +
+residual), inputs resident in HBM.  Default workload: the bf16 model-shaped
+one (B=4, T=2048, 16 heads x 64 = 1024-d e_t, H=1024, hc=4).
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
+the launching stream; L2 is flushed (256 MB write) between steps outside the
+events; barrier + synchronize on both sides; the max over ranks is reported.
+Multi-GPU: one process per GPU, every rank runs its own replica of the
+workload (the pass has no cross-sequence exchange), scaling "weak".
+
+The dominant kernel (the projection) is timed by CUDA events the library
+records at its stage boundaries (engram_set_stage_events).  The CPU baseline is
+the float64 oracle on a bounded sample of the same workload on the host cores.
+
+--impl reference runs that oracle as the reference arm (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except OSError:
+        return PEAKS_FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        # nvidia-smi numbers GPUs physically; address this one by its UUID
+        try:
+            self.index = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            ids = [x for x in vis.split(",") if x.strip()]
+            self.index = ids[device_index] if device_index < len(ids) else str(device_index)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.index, "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    sm.append(float(parts[2]))
+                    smax.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[6:10]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle (CPU)
+def oracle_sample(w, tokens: int, nthreads: int):
+    """Prepare the float64 oracle over the first `tokens` positions of
+    sequence 0 of a workload of the same shapes and distributions (whole pass
+    from ids, host cores).  Returns (n, run) where run() -> seconds."""
+    from hashed_gram_conditional_hash_b200 import workloads as W
+    from oracle import engram_oracle as O
+    n = max(1, min(tokens, w.seq_len))
+    if W.gen_device_for(w, "cuda") == "cpu":
+        wp = w.replace(B=1, T=n, decode_calls=0)
+        p = W.make_params(wp, "cpu")
+        x = p.ids.numpy()
+        if p.lookup is not None:
+            x = O.compress_ids(x, p.lookup.numpy())
+
+        def run():
+            t0 = time.perf_counter()
+            O.forward(x=x, orders=wp.orders, J=wp.heads_per_order, mult=p.mult, primes=p.primes,
+                      row_offsets=p.offsets, pad_id=wp.pad_id, table=p.table, w_value=p.w_value,
+                      w_key=p.w_key, norm_key=p.norm_key, norm_query=p.norm_query,
+                      conv_w=p.conv_w, hidden=p.hidden, K=wp.conv_kernel, dil=wp.dil,
+                      nthreads=nthreads)
+            return time.perf_counter() - t0
+        return n, run
+    # tables drawn on the device: the oracle receives the rows it needs
+    p = W.make_params(w, "cuda")
+    dev = p.table.device
+    pos = [(0, t) for t in range(n)]
+    if w.decode_calls:
+        hid = lambda b, t: p.hidden[torch.from_numpy(t).to(dev), torch.from_numpy(b).to(dev)].cpu()
+    else:
+        hid = lambda b, t: p.hidden[torch.from_numpy(b).to(dev), torch.from_numpy(t).to(dev)].cpu()
+    x = p.ids.cpu().numpy()
+    args = (p.w_value.cpu(), p.w_key.cpu(), p.norm_key.cpu(), p.norm_query.cpu(), p.conv_w.cpu())
+
+    def run():
+        t0 = time.perf_counter()
+        O.forward_sampled(x, pos, w.orders, w.heads_per_order, p.mult, p.primes, p.offsets,
+                          w.pad_id, lambda r: p.table[torch.from_numpy(r).to(dev)].cpu(), hid,
+                          *args, K=w.conv_kernel, dil=w.dil, nthreads=nthreads)
+        return time.perf_counter() - t0
+    return n, run
+
+
+def oracle_tokens_for(w, seconds: float, nthreads: int) -> int:
+    """Sample size that takes about `seconds` of oracle time (calibrated)."""
+    n, run = oracle_sample(w, 32, nthreads)
+    run()
+    dt = run()
+    return int(max(8, n / max(dt, 1e-6) * seconds))
+
+
+def cpu_baseline(w, budget_s: float):
+    nthreads = os.cpu_count() or 1
+    n, run = oracle_sample(w, oracle_tokens_for(w, budget_s, nthreads), nthreads)
+    dt = run()
+    return {"value": n / dt, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "sample": "first %d positions of sequence 0 of workload %s (same shapes and "
+                      "distributions), whole pass from ids, float64, %.1f s" % (n, w.name, dt)}
+
+
+# ---------------------------------------------------------------- GPU arm
+def algorithmic(w):
+    """Per-token algorithmic bytes / flops of each stage (see the design notes)."""
+    es = w.elem_bytes
+    return {
+        "proj_flops": 2.0 * w.E * w.hidden * (1 + w.hc_mult),
+        "hash_bytes": 8.0 + 4.0 * w.nh,                      # ids in, int32 rows out
+        "gather_bytes": float(w.E * es),                     # rows read once
+        "conv_bytes": float(w.hidden * es + 4 * w.hc_mult + w.hc_mult * w.hidden * es),
+        "pass_bytes": float(8 + w.E * es + 2 * w.hc_mult * w.hidden * es),
+    }
+
+
+def run_ours(args, rank, world, device):
+    from hashed_gram_conditional_hash_b200 import EngramLayer
+    from hashed_gram_conditional_hash_b200 import _lib as L
+    from hashed_gram_conditional_hash_b200 import workloads as W
+
+    w = W.CONFIGS[args.config]
+    peaks, peak_kind = load_peaks()
+    p = W.make_params(w, device)
+    layer = EngramLayer.from_params(p)
+    engine = "tcgen05" if L.engram_projection_engine(layer.cfg) == L.ENGINE_TCGEN05 else "simt"
+    stream = torch.cuda.current_stream()
+    decode = bool(w.decode_calls)
+    if decode:
+        Bq, Tq = w.B, 1
+        state = layer.new_state(w.B)
+        steps_ids = p.ids.t().contiguous().view(w.decode_calls, w.B, 1)
+        step_in = lambda i: (steps_ids[i % w.decode_calls],
+                             p.hidden[i % w.decode_calls].view(w.B, 1, w.hc_mult, w.hidden))
+    else:
+        Bq, Tq = w.B, w.T
+        state = None
+        step_in = lambda i: (p.ids, p.hidden)
+    ws = layer.workspace(Bq, Tq)
+    y = torch.empty((Bq, Tq, w.hc_mult, w.hidden), dtype=w.torch_dtype, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def step(i):
+        ids, hid = step_in(i)
+        layer.forward(ids, hid, y=y, ws=ws, state=state, dev_status=st)
+
+    for i in range(args.warmup):
+        step(i)
+        flush.fill_(i & 0xff)
+    torch.cuda.synchronize()
+    bits = L.engram_read_status(st)
+    if bits:
+        raise RuntimeError("device status 0x%x during warm-up" % bits)
+
+    K = args.steps
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [{k: mk() for k in ("before_hash", "before_projection", "before_gate", "before_conv",
+                             "after_conv")} for _ in range(K)]
+    for e in ev:  # create the underlying events before handing them to the library
+        for x in e.values():
+            x.record(stream)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    n0 = L.engram_launch_count()
+    for i in range(K):
+        L.engram_set_stage_events(ev[i])
+        step(args.warmup + i)
+        L.engram_set_stage_events(None)
+        flush.fill_(i & 0xff)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = L.engram_launch_count() - n0
+    clk = clocks.stop() if clocks else None
+    bits = L.engram_read_status(st)
+    if bits:
+        raise RuntimeError("device status 0x%x during the timed steps" % bits)
+
+    t_step = sum(e["before_hash"].elapsed_time(e["after_conv"]) for e in ev)       # ms
+    t_proj = sum(e["before_projection"].elapsed_time(e["before_gate"]) for e in ev)
+    t_hash = sum(e["before_hash"].elapsed_time(e["before_projection"]) for e in ev)
+    t_gate = sum(e["before_gate"].elapsed_time(e["before_conv"]) for e in ev)
+    t_conv = sum(e["before_conv"].elapsed_time(e["after_conv"]) for e in ev)
+    times = torch.tensor([t_step, t_proj, t_hash, t_gate, t_conv], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    t_step, t_proj, t_hash, t_gate, t_conv = times.tolist()
+
+    tokens_step = Bq * Tq
+    value = world * tokens_step * K / (t_step / 1e3)
+    a = algorithmic(w)
+    proj_s = t_proj / K / 1e3
+    proj_tflops = a["proj_flops"] * tokens_step / proj_s / 1e12
+    tc_peak = peaks["bf16_tflops"]
+    stages = {
+        "hash": {"us": t_hash / K * 1e3, "bound": "hbm",
+                 "achieved_gbs": a["hash_bytes"] * tokens_step / (t_hash / K / 1e3) / 1e9},
+        "projection": {"us": t_proj / K * 1e3, "bound": "tensor", "engine": engine,
+                       "achieved_tflops": proj_tflops},
+        "gate": {"us": t_gate / K * 1e3},
+        "conv": {"us": t_conv / K * 1e3, "bound": "hbm",
+                 "achieved_gbs": a["conv_bytes"] * tokens_step / (t_conv / K / 1e3) / 1e9},
+    }
+    for s in ("hash", "conv"):
+        stages[s]["frac_of_measured_hbm"] = stages[s]["achieved_gbs"] / peaks["hbm_gbs"]
+    result = {
+        "metric": "Engram forward tokens/s on 1xB200 (engram_forward); % of HBM and bf16 tensor roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": t_step / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded; shapes and distributions of the workload)",
+        "config": {"workload": w.name, "B": w.B, "T": Tq, "tokens_per_step_per_gpu": tokens_step,
+                   "orders": list(w.orders), "heads_per_order": w.heads_per_order,
+                   "row_dim": w.row_dim, "hidden": w.hidden, "hc_mult": w.hc_mult,
+                   "dilation": w.dil, "table_gb": round(W.table_bytes(w) / 1e9, 3),
+                   "l2": "flushed (256 MB write) between timed steps",
+                   "parallelism": "replicas x%d" % world, "projection_engine": engine},
+        "roofline": {"bound": "tensor", "kernel": "proj_tc_kernel" if engine == "tcgen05" else "proj_simt_kernel",
+                     "achieved": proj_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": proj_tflops / tc_peak, "peak_kind": "%s bf16 burst" % peak_kind,
+                     "traffic": None,
+                     "flops_per_launch": a["proj_flops"] * tokens_step},
+        "stages": stages,
+        "clocks": clk,
+        "gpu_launches": int(launches),
+    }
+    return result, layer, p, w
+
+
+def run_e2e(args, layer, p, w, device, world):
+    """Same metric through the public API with host buffers: pinned ids and
+    hidden states copied in, y copied out, every step inside the events."""
+    decode = bool(w.decode_calls)
+    if decode:
+        Bq, Tq = w.B, 1
+        ids_h = p.ids[:, :1].contiguous().cpu().pin_memory()
+        hid_h = p.hidden[0].view(w.B, 1, w.hc_mult, w.hidden).cpu().pin_memory()
+        state = layer.new_state(w.B)
+    else:
+        Bq, Tq = w.B, w.T
+        ids_h = p.ids.cpu().pin_memory()
+        hid_h = p.hidden.cpu().pin_memory()
+        state = None
+    y_h = torch.empty((Bq, Tq, w.hc_mult, w.hidden), dtype=w.torch_dtype).pin_memory()
+    ids_d = torch.empty_like(ids_h, device=device)
+    hid_d = torch.empty_like(hid_h, device=device)
+    y_d = torch.empty_like(y_h, device=device)
+    ws = layer.workspace(Bq, Tq)
+
+    def step():
+        ids_d.copy_(ids_h, non_blocking=True)
+        hid_d.copy_(hid_h, non_blocking=True)
+        layer.forward(ids_d, hid_d, y=y_d, ws=ws, state=state)
+        y_h.copy_(y_d, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    K = max(3, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(K):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = t.item()
+    h2d = ids_h.numel() * 8 + hid_h.numel() * hid_h.element_size()
+    d2h = y_h.numel() * y_h.element_size()
+    return {"value": world * Bq * Tq * K / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def run_reference(args):
+    """The reference arm: the float64 oracle on the host cores, K timed steps
+    of a bounded sample each, sized so that warm-up + steps take ~2 minutes."""
+    from hashed_gram_conditional_hash_b200 import workloads as W
+    w = W.CONFIGS[args.config]
+    nthreads = os.cpu_count() or 1
+    per_step = min(args.ref_step_s, 120.0 / max(1, args.steps + args.warmup))
+    n, run = oracle_sample(w, oracle_tokens_for(w, per_step, nthreads), nthreads)
+    for _ in range(args.warmup):
+        run()
+    tot = 0.0
+    for _ in range(args.steps):
+        tot += run()
+    rate = n * args.steps / tot
+    sample = ("per step: first %d positions of sequence 0 of workload %s (same shapes and "
+              "distributions), whole pass from ids, float64 oracle" % (n, w.name))
+    return {
+        "impl": "reference",
+        "metric": "Engram forward tokens/s on 1xB200 (engram_forward); % of HBM and bf16 tensor roofline",
+        "value": rate, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "B": w.B, "T": w.T if not w.decode_calls else 1},
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="model_bf16")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--ref-step-s", type=float, default=3.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    device = "cuda:%d" % local
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device(device))
+    try:
+        res, layer, p, w = run_ours(args, rank, world, device)
+        if not args.no_e2e:
+            res["e2e"] = run_e2e(args, layer, p, w, device, world)
+        del layer, p
+        torch.cuda.empty_cache()
+        if rank == 0 and not args.no_cpu_baseline and world == 1:
+            res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget_s)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

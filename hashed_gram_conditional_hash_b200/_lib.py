@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libengram.so")
 MAX_ORDERS = 8
 ENGRAM_F32, ENGRAM_BF16 = 0, 1
 STATUS_ID_RANGE, STATUS_ROW_RANGE, STATUS_TIMEOUT = 0x1, 0x2, 0x4
-DEBUG_FORCE_TIMEOUT, DEBUG_FORCE_SIMT = 0x1, 0x2
+DEBUG_FORCE_TIMEOUT, DEBUG_FORCE_SIMT, DEBUG_FUSED_GATHER = 0x1, 0x2, 0x4
 STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_CUDA",
                 4: "ERR_TIMEOUT", 5: "ERR_ID_RANGE"}
 
@@ -50,6 +50,12 @@ class EngramWeights(C.Structure):
                 ("norm_key", C.c_void_p), ("norm_query", C.c_void_p), ("conv_w", C.c_void_p)]
 
 
+class EngramStageEvents(C.Structure):
+    _fields_ = [("before_hash", C.c_void_p), ("before_projection", C.c_void_p),
+                ("before_gate", C.c_void_p), ("before_conv", C.c_void_p),
+                ("after_conv", C.c_void_p)]
+
+
 class EngramState(C.Structure):
     _fields_ = [("id_ring", C.c_void_p), ("v_ring", C.c_void_p), ("g_ring", C.c_void_p),
                 ("pos", C.c_void_p), ("ring_len", C.c_int32)]
@@ -75,6 +81,8 @@ def lib() -> C.CDLL:
             "engram_read_status": (C.c_int, [P, P, P]),
             "engram_set_debug": (None, [C.c_uint32]),
             "engram_projection_engine": (i32, [cfg]),
+            "engram_launch_count": (C.c_uint64, []),
+            "engram_set_stage_events": (None, [C.POINTER(EngramStageEvents)]),
             "engram_compress_ids": (C.c_int, [P, i64, P, i64, P, P, P]),
             "engram_hash": (C.c_int, [cfg, P, i32, i32, P, P, P, P, P, P]),
             "engram_gather": (C.c_int, [cfg, P, i64, P, P, i64, P, P, P]),
@@ -158,8 +166,23 @@ def engram_version() -> int:
     return lib().engram_version()
 
 
+def engram_launch_count() -> int:
+    return lib().engram_launch_count()
+
+
 def engram_set_debug(flags: int) -> None:
     lib().engram_set_debug(flags)
+
+
+def engram_set_stage_events(events: Optional[dict]) -> None:
+    """events: {stage name: torch.cuda.Event (already recorded once)} or None."""
+    if events is None:
+        lib().engram_set_stage_events(None)
+        return
+    ev = EngramStageEvents()
+    for k, e in events.items():
+        setattr(ev, k, e.cuda_event)
+    lib().engram_set_stage_events(C.byref(ev))
 
 
 ENGINE_SIMT, ENGINE_TCGEN05 = 0, 1

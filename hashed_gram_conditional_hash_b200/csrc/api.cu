@@ -14,6 +14,13 @@ namespace {
 
 thread_local char g_err[512] = "";
 std::atomic<uint32_t> g_debug{0};
+engram_stage_events g_events = {nullptr, nullptr, nullptr, nullptr, nullptr};
+std::atomic<bool> g_events_on{false};
+
+void record(void* ev, cudaStream_t s) {
+  if (ev != nullptr && g_events_on.load(std::memory_order_relaxed))
+    cudaEventRecord(static_cast<cudaEvent_t>(ev), s);
+}
 
 engram_status fail(engram_status st, const char* fmt, ...) {
   va_list ap;
@@ -122,15 +129,23 @@ StageLayout stage_layout(const engram_config* c, int64_t M, size_t start) {
 
 int64_t rows_ld(int64_t M) { return (M + 127) / 128 * 128; }
 
+// Forward workspace: either (idx [M, nh] int64, e [M, E]) for the gather-then-
+// project path, or the head-major int32 rows [nh, rows_ld(M)] of the fused
+// path, in one shared region; then V, partials and gates.
 struct ForwardLayout {
-  size_t rows_off;
+  size_t idx_off, e_off, rows_off;
   StageLayout st;
 };
 ForwardLayout forward_layout(const engram_config* c, int64_t M) {
   ForwardLayout L;
-  L.rows_off = 0;
   const int nh = c->n_orders * c->heads_per_order;
-  L.st = stage_layout(c, M, static_cast<size_t>(nh) * rows_ld(M) * sizeof(int32_t));
+  const size_t es = c->dtype == ENGRAM_F32 ? 4 : 2;
+  L.idx_off = 0;
+  L.e_off = align256(static_cast<size_t>(M) * nh * sizeof(int64_t));
+  const size_t split_end = align256(L.e_off + static_cast<size_t>(M) * nh * c->row_dim * es);
+  L.rows_off = 0;
+  const size_t rows_end = align256(static_cast<size_t>(nh) * rows_ld(M) * sizeof(int32_t));
+  L.st = stage_layout(c, M, split_end > rows_end ? split_end : rows_end);
   return L;
 }
 
@@ -139,14 +154,23 @@ bool use_tc(const engram_config* c) {
   return tc_projection_supported(c->row_dim, c->hidden, c->dtype);
 }
 
-// The projection + gate stage shared by engram_forward and engram_gate_fuse.
+// The projection stage shared by engram_forward and engram_gate_fuse; sets
+// pp->n_tiles to the partials granularity of the engine that ran.
+engram_status run_projection(const engram_config* c, ProjParams* pp, cudaStream_t s) {
+  const bool tc = use_tc(c);
+  pp->n_tiles = c->hidden / (tc ? kTcTileN : kSimtTileN);
+  pp->debug = g_debug.load();
+  record(g_events.before_projection, s);
+  engram_status st = tc ? cuda_check(launch_proj_tc(*pp, s), "projection (tcgen05)")
+                        : cuda_check(launch_proj_simt(*pp, s), "projection (SIMT)");
+  record(g_events.before_gate, s);
+  return st;
+}
+
+// Projection followed by the stand-alone gate kernel (engram_gate_fuse).
 engram_status run_stage(const engram_config* c, ProjParams pp, float* g, float* g_copy,
                         cudaStream_t s) {
-  const bool tc = use_tc(c);
-  pp.n_tiles = c->hidden / (tc ? kTcTileN : kSimtTileN);
-  pp.debug = g_debug.load();
-  engram_status st = tc ? cuda_check(launch_proj_tc(pp, s), "projection (tcgen05)")
-                        : cuda_check(launch_proj_simt(pp, s), "projection (SIMT)");
+  engram_status st = run_projection(c, &pp, s);
   if (st != ENGRAM_OK) return st;
   GateParams gp;
   gp.partials = pp.partials;
@@ -162,6 +186,12 @@ engram_status run_stage(const engram_config* c, ProjParams pp, float* g, float* 
 }
 
 }  // namespace
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 int num_sms() {
   static int cache[64] = {0};
@@ -195,6 +225,18 @@ size_t engram_last_error(char* buf, size_t n) {
 }
 
 void engram_set_debug(uint32_t flags) { g_debug.store(flags); }
+
+uint64_t engram_launch_count(void) { return g_launches.load(); }
+
+void engram_set_stage_events(const engram_stage_events* events) {
+  if (events == nullptr) {
+    g_events_on.store(false);
+    g_events = engram_stage_events{nullptr, nullptr, nullptr, nullptr, nullptr};
+  } else {
+    g_events = *events;
+    g_events_on.store(true);
+  }
+}
 
 int32_t engram_projection_engine(const engram_config* cfg) {
   if (check_config(cfg) != ENGRAM_OK) return -1;
@@ -441,29 +483,51 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   char* w = static_cast<char*>(ws);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  // a1-a3: ids -> absolute table rows (head-major)
+  // a1-a3: ids -> hash indices (or absolute table rows for the fused path)
+  const bool fused = (g_debug.load() & ENGRAM_DEBUG_FUSED_GATHER) != 0;
   const int64_t ld = rows_ld(M);
   int32_t* rows = reinterpret_cast<int32_t*>(w + L.rows_off);
+  int64_t* idx = reinterpret_cast<int64_t*>(w + L.idx_off);
+  void* e = w + L.e_off;
   hp.ids = ids;
   hp.lookup = wts->lookup;
   hp.raw_vocab = wts->raw_vocab;
   hp.history = state != nullptr ? state->id_ring : nullptr;
   hp.id_ring_out = state != nullptr ? state->id_ring : nullptr;
-  hp.rows_out = rows;
+  hp.rows_out = fused ? rows : nullptr;
+  hp.idx_out = fused ? nullptr : idx;
   hp.ld_rows = ld;
   hp.status = dev_status;
   hp.B = B;
   hp.T = T;
+  record(g_events.before_hash, s);
   st = cuda_check(launch_hash(hp, s), "hash");
   if (st != ENGRAM_OK) return st;
 
-  // a4-a7: gathered projection, score partials, gates
+  // a4: e = the gathered rows, once (unless fused into the projection)
+  if (!fused) {
+    GatherParams gp;
+    memset(&gp, 0, sizeof gp);
+    gp.table = wts->table;
+    gp.idx = idx;
+    gp.e = e;
+    gp.status = dev_status;
+    gp.M = M;
+    gp.total_rows = wts->total_rows;
+    gp.nh = hp.nh;
+    gp.row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
+    for (int h = 0; h < hp.nh; ++h) gp.row_off[h] = hp.row_off[h];
+    st = cuda_check(launch_gather(gp, s), "gather");
+    if (st != ENGRAM_OK) return st;
+  }
+
+  // a5-a7: projection, score partials, gates
   ProjParams pp;
   memset(&pp, 0, sizeof pp);
-  pp.a_src = wts->table;
-  pp.rows = rows;
+  pp.a_src = fused ? wts->table : e;
+  pp.rows = fused ? rows : nullptr;
   pp.ld_rows = ld;
-  pp.a_rows = wts->total_rows;
+  pp.a_rows = fused ? wts->total_rows : M * hp.nh;
   pp.w_value = wts->w_value;
   pp.w_key = wts->w_key;
   pp.norm_key = wts->norm_key;
@@ -503,7 +567,9 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   cp.K = cfg->conv_kernel;
   cp.dil = cfg->dilation;
   cp.dtype = cfg->dtype;
+  record(g_events.before_conv, s);
   st = cuda_check(launch_gated_conv(cp, s), "gated conv");
+  record(g_events.after_conv, s);
   if (st != ENGRAM_OK || state == nullptr) return st;
 
   StateAdvanceParams ap;

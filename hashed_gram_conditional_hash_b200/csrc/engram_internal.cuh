@@ -7,7 +7,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/engram.h"
+#include "engram.h"  // include/ is on the include path
 
 namespace engram {
 
@@ -80,7 +80,7 @@ struct ProjParams {
 };
 // Column-tile widths of the two projection engines (partials granularity).
 constexpr int kSimtTileN = 64;
-constexpr int kTcTileN = 256;
+constexpr int kTcTileN = 128;
 bool tc_projection_supported(int Dh, int H, engram_dtype dt);
 cudaError_t launch_proj_simt(const ProjParams& p, cudaStream_t s);
 cudaError_t launch_proj_tc(const ProjParams& p, cudaStream_t s);
@@ -96,7 +96,7 @@ struct GateParams {
 };
 cudaError_t launch_gate(const GateParams& p, cudaStream_t s);
 
-// Gated value + short conv + residual (a8, a9) from V and g.
+// Gated value + short conv + residual (a8, a9) from V and the gates.
 //   Y[b,t,h,c] = U(t) + sum_i w[h*H+c, i] U(t - (K-1-i) dil),  U(t) = g[t,h] V[t,c]
 // Positions before the chunk come from the state rings (if any) or are zero.
 // conv_w == null: Y = U (no conv; used by engram_gate_fuse).
@@ -144,6 +144,9 @@ cudaError_t launch_state_init(int64_t* id_ring, int n_hist, void* v_ring, float*
 // Number of SMs of the current device (cached per device).
 int num_sms();
 
+// Count of kernels launched by the library (engram_launch_count).
+void count_launch(int n = 1);
+
 // ---------------------------------------------------------------- device side
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
@@ -175,9 +178,9 @@ template <> struct Elem<uint16_t> {
 };
 
 // Exact x mod p for x < 2^64, p >= 2, with mu = floor((2^64 - 1) / p)
-// (Barrett reduction: the estimate q = floor(x * mu / 2^64) is at most one
-// below floor(x / p), so one conditional subtraction suffices; a second is
-// kept for safety).
+// (Barrett reduction: the estimate q = floor(x * mu / 2^64) never exceeds
+// floor(x / p) and is at most two below it, so two conditional subtractions
+// give the exact remainder; for the x < 2^63 the hash produces, one suffices).
 __device__ __forceinline__ uint64_t barrett_mod(uint64_t x, uint64_t p, uint64_t mu) {
   uint64_t q = __umul64hi(x, mu);
   uint64_t r = x - q * p;

@@ -24,7 +24,15 @@ __global__ void gate_kernel(const __grid_constant__ GateParams p) {
   if (i >= p.M * p.hc) return;
   const float4* part = p.partials + i * p.n_tiles;
   float dot = 0.f, ssk = 0.f, ssq = 0.f;
-  for (int t = 0; t < p.n_tiles; ++t) {
+  int t = 0;
+  for (; t + 8 <= p.n_tiles; t += 8) {   // eight independent loads in flight
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldg(part + t + u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) { dot += v[u].x; ssk += v[u].y; ssq += v[u].z; }
+  }
+  for (; t < p.n_tiles; ++t) {
     const float4 v = __ldg(part + t);
     dot += v.x;
     ssk += v.y;
@@ -40,79 +48,147 @@ __global__ void gate_kernel(const __grid_constant__ GateParams p) {
 }
 
 // -------------------------------------------------------------- gated conv
-template <typename T> struct Pair;
-template <> struct Pair<float> {
-  static __device__ __forceinline__ float2 load(const float* base, int64_t i) {
-    return __ldg(reinterpret_cast<const float2*>(base + i));
+// Eight consecutive channels of one row as floats.
+template <typename T> struct Vec8;
+template <> struct Vec8<uint16_t> {
+  static __device__ __forceinline__ void load(const uint16_t* p, float (&v)[8]) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(u[i] << 16);
+      v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
   }
-  static __device__ __forceinline__ void store(float* base, int64_t i, float2 v) {
-    *reinterpret_cast<float2*>(base + i) = v;
+  static __device__ __forceinline__ void store(uint16_t* p, const float (&v)[8]) {
+    uint4 w;
+    w.x = static_cast<uint32_t>(f32_to_bf16(v[0])) | (static_cast<uint32_t>(f32_to_bf16(v[1])) << 16);
+    w.y = static_cast<uint32_t>(f32_to_bf16(v[2])) | (static_cast<uint32_t>(f32_to_bf16(v[3])) << 16);
+    w.z = static_cast<uint32_t>(f32_to_bf16(v[4])) | (static_cast<uint32_t>(f32_to_bf16(v[5])) << 16);
+    w.w = static_cast<uint32_t>(f32_to_bf16(v[6])) | (static_cast<uint32_t>(f32_to_bf16(v[7])) << 16);
+    *reinterpret_cast<uint4*>(p) = w;
   }
 };
-template <> struct Pair<uint16_t> {
-  static __device__ __forceinline__ float2 load(const uint16_t* base, int64_t i) {
-    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(base + i));
-    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+template <> struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   }
-  static __device__ __forceinline__ void store(uint16_t* base, int64_t i, float2 v) {
-    const uint32_t w = static_cast<uint32_t>(f32_to_bf16(v.x)) |
-                       (static_cast<uint32_t>(f32_to_bf16(v.y)) << 16);
-    *reinterpret_cast<uint32_t*>(base + i) = w;
+  static __device__ __forceinline__ void store(float* p, const float (&v)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
   }
 };
 
-template <typename T>
-__global__ void __launch_bounds__(256) gated_conv_kernel(const __grid_constant__ ConvParams p,
-                                                         int tile_t) {
-  const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 2;
-  if (c >= p.H) return;
-  const int b = blockIdx.z;
-  const int t0 = blockIdx.y * tile_t;
-  const int t1 = min(t0 + tile_t, p.T);
+constexpr int kConvThreads = 256;
+
+// Conv taps of 8 consecutive channels: w[j][i] = row[j*K + i] (8K contiguous
+// values); 16-byte loads when K == 4.
+template <typename T, int KMAX>
+__device__ __forceinline__ void load_taps(const T* row, int K, float (&w)[8][KMAX]) {
+  if (K == 4 && KMAX >= 4) {
+    if (sizeof(T) == 2) {
+      const uint4* q = reinterpret_cast<const uint4*>(row);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint4 x = __ldg(q + u);
+        const uint32_t a[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {   // values 8u + 2e, 8u + 2e + 1
+          const int k0 = 8 * u + 2 * e;
+          w[k0 / 4][k0 % 4] = __uint_as_float(a[e] << 16);
+          w[(k0 + 1) / 4][(k0 + 1) % 4] = __uint_as_float(a[e] & 0xffff0000u);
+        }
+      }
+    } else {
+      const float4* q = reinterpret_cast<const float4*>(row);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 x = __ldg(q + j);
+        w[j][0] = x.x; w[j][1] = x.y; w[j][2] = x.z; w[j][3] = x.w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int i = 4; i < KMAX; ++i) w[j][i] = 0.f;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int i = 0; i < KMAX; ++i) w[j][i] = i < K ? Elem<T>::load(row, j * K + i) : 0.f;
+  }
+}
+
+// One thread per (position, 8 consecutive channels), all branches: it loads
+// the K value taps and their gates (independent loads; neighbouring
+// positions re-read the same rows from L1/L2), then for every branch the 8K
+// conv taps (one contiguous run of the weight matrix) and writes 8 channels
+// of Y.  Every load of a thread is independent of the others, so the kernel
+// keeps many bytes in flight and runs at the memory system's pace.
+template <typename T, int KMAX, int HCMAX>
+__global__ void __launch_bounds__(kConvThreads) gated_conv_kernel(const __grid_constant__ ConvParams p) {
+  const int cgs = p.H >> 3;                                   // channel groups per row
+  const int64_t gid = blockIdx.x * static_cast<int64_t>(kConvThreads) + threadIdx.x;
+  const int64_t row = gid / cgs;                              // token b*T + t
+  if (row >= static_cast<int64_t>(p.B) * p.T) return;
+  const int c = static_cast<int>(gid - row * cgs) * 8;
+  const int b = static_cast<int>(row / p.T);
+  const int t = static_cast<int>(row - static_cast<int64_t>(b) * p.T);
   const T* V = static_cast<const T*>(p.V);
   const T* W = static_cast<const T*>(p.conv_w);
   const T* vr = static_cast<const T*>(p.v_ring);
   T* Y = static_cast<T*>(p.Y);
-  const int64_t seq = static_cast<int64_t>(b) * p.T;
+  const int K = (W != nullptr) ? p.K : 1;                     // no conv: only U(t)
   const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) : 0;
 
-  for (int h = 0; h < p.hc; ++h) {
-    float2 w[ENGRAM_MAX_CONV_K];
+  // the position itself
+  float vt[8], gt[HCMAX];
+  Vec8<T>::load(V + row * p.H + c, vt);
 #pragma unroll
-    for (int i = 0; i < ENGRAM_MAX_CONV_K; ++i) {
-      w[i] = make_float2(0.f, 0.f);
-      if (W != nullptr && i < p.K) {
-        const int64_t r = static_cast<int64_t>(h) * p.H + c;
-        w[i].x = Elem<T>::load(W, r * p.K + i);
-        w[i].y = Elem<T>::load(W, (r + 1) * p.K + i);
-      }
+  for (int h = 0; h < HCMAX; ++h) gt[h] = h < p.hc ? __ldg(p.g + row * p.hc + h) : 0.f;
+  // taps i = 0 .. K-1 at positions t - (K-1-i)*dil (tap K-1 is t itself)
+  float v[KMAX][8];
+  float g[KMAX][HCMAX];
+#pragma unroll
+  for (int i = 0; i < KMAX; ++i) {
+    const int d = (K - 1 - i) * p.dil;
+    const int tp = t - d;
+    const bool in_seq = i < K && tp >= 0;
+    const bool in_ring = i < K && tp < 0 && vr != nullptr && P + tp >= 0;
+    int64_t rb = 0;
+    if (in_ring) rb = static_cast<int64_t>(b) * p.ring_len + (P + tp) % p.ring_len;
+    const float* gsrc = in_seq ? p.g + (row - d) * p.hc : p.g_ring + rb * p.hc;
+    const T* vsrc = in_seq ? V + (row - d) * p.H + c : vr + rb * p.H + c;
+    if (in_seq || in_ring) {
+      Vec8<T>::load(vsrc, v[i]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[i][j] = 0.f;
     }
-    for (int t = t0; t < t1; ++t) {
-      // U(t) itself
-      const float gt = __ldg(p.g + (seq + t) * p.hc + h);
-      const float2 vt = Pair<T>::load(V, (seq + t) * p.H + c);
-      float2 acc = make_float2(gt * vt.x, gt * vt.y);
-      if (W != nullptr) {
 #pragma unroll
-        for (int i = 0; i < ENGRAM_MAX_CONV_K; ++i) {
-          if (i >= p.K) break;
-          const int tp = t - (p.K - 1 - i) * p.dil;
-          float gp = 0.f;
-          float2 vp = make_float2(0.f, 0.f);
-          if (tp >= 0) {
-            gp = __ldg(p.g + (seq + tp) * p.hc + h);
-            vp = Pair<T>::load(V, (seq + tp) * p.H + c);
-          } else if (vr != nullptr && P + tp >= 0) {
-            const int64_t slot = (P + tp) % p.ring_len;
-            const int64_t rb = static_cast<int64_t>(b) * p.ring_len + slot;
-            gp = __ldg(p.g_ring + rb * p.hc + h);
-            vp = Pair<T>::load(vr, rb * p.H + c);
-          }
-          acc.x = fmaf(w[i].x, gp * vp.x, acc.x);
-          acc.y = fmaf(w[i].y, gp * vp.y, acc.y);
-        }
+    for (int h = 0; h < HCMAX; ++h)
+      g[i][h] = ((in_seq || in_ring) && h < p.hc) ? __ldg(gsrc + h) : 0.f;
+  }
+#pragma unroll
+  for (int h = 0; h < HCMAX; ++h) {
+    if (h < p.hc) {
+      // U(t) itself
+      float acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = gt[h] * vt[j];
+      if (W != nullptr) {
+        // weights of channels h*H + c .. +7, taps 0 .. K-1: 8K contiguous values
+        float w[8][KMAX];
+        load_taps<T, KMAX>(W + (static_cast<int64_t>(h) * p.H + c) * p.K, p.K, w);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+          for (int i = 0; i < KMAX; ++i) acc[j] = fmaf(w[j][i], g[i][h] * v[i][j], acc[j]);
       }
-      Pair<T>::store(Y, ((seq + t) * p.hc + h) * p.H + c, acc);
+      Vec8<T>::store(Y + (row * p.hc + h) * p.H + c, acc);
     }
   }
 }
@@ -207,21 +283,27 @@ cudaError_t launch_gate(const GateParams& p, cudaStream_t s) {
   const int64_t n = p.M * p.hc;
   if (n <= 0) return cudaSuccess;
   gate_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
+  count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
   if (p.B <= 0 || p.T <= 0) return cudaSuccess;
-  const int threads = 256;
-  const int cblocks = (p.H / 2 + threads - 1) / threads;
-  // sequence tile: as long as possible (less halo re-read) while keeping at
-  // least ~4 blocks per SM resident
-  const int64_t want = static_cast<int64_t>(num_sms()) * 4;
-  int tile = 64;
-  while (tile > 4 && static_cast<int64_t>(cblocks) * p.B * ((p.T + tile - 1) / tile) < want) tile >>= 1;
-  dim3 grid(cblocks, (p.T + tile - 1) / tile, p.B);
-  if (p.dtype == ENGRAM_F32) gated_conv_kernel<float><<<grid, threads, 0, s>>>(p, tile);
-  else gated_conv_kernel<uint16_t><<<grid, threads, 0, s>>>(p, tile);
+  if (p.H % 8 != 0) return cudaErrorInvalidValue;
+  const int64_t threads = static_cast<int64_t>(p.B) * p.T * (p.H / 8);
+  const int64_t blocks = (threads + kConvThreads - 1) / kConvThreads;
+  if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+  const unsigned nb = static_cast<unsigned>(blocks);
+  if (p.K <= 4 && p.hc <= 4) {  // the pages' shape: kernel 4, up to 4 branches
+    if (p.dtype == ENGRAM_F32) gated_conv_kernel<float, 4, 4><<<nb, kConvThreads, 0, s>>>(p);
+    else gated_conv_kernel<uint16_t, 4, 4><<<nb, kConvThreads, 0, s>>>(p);
+  } else {
+    if (p.dtype == ENGRAM_F32)
+      gated_conv_kernel<float, ENGRAM_MAX_CONV_K, ENGRAM_MAX_HC><<<nb, kConvThreads, 0, s>>>(p);
+    else
+      gated_conv_kernel<uint16_t, ENGRAM_MAX_CONV_K, ENGRAM_MAX_HC><<<nb, kConvThreads, 0, s>>>(p);
+  }
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -232,6 +314,7 @@ cudaError_t launch_short_conv(const ShortConvParams& p, cudaStream_t s) {
     if (blocks > grid_cap()) blocks = grid_cap();
     if (p.dtype == ENGRAM_F32) short_conv_kernel<float><<<static_cast<int>(blocks), 256, 0, s>>>(p);
     else short_conv_kernel<uint16_t><<<static_cast<int>(blocks), 256, 0, s>>>(p);
+    count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -240,6 +323,7 @@ cudaError_t launch_short_conv(const ShortConvParams& p, cudaStream_t s) {
     const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
     if (p.dtype == ENGRAM_F32) short_conv_state_kernel<float><<<blocks, 256, 0, s>>>(p);
     else short_conv_state_kernel<uint16_t><<<blocks, 256, 0, s>>>(p);
+    count_launch();
     return cudaGetLastError();
   }
   return cudaSuccess;
@@ -249,6 +333,7 @@ cudaError_t launch_state_advance(const StateAdvanceParams& p, cudaStream_t s) {
   if (p.B <= 0 || p.T <= 0) return cudaSuccess;
   if (p.dtype == ENGRAM_F32) state_advance_kernel<float><<<p.B, 256, 0, s>>>(p);
   else state_advance_kernel<uint16_t><<<p.B, 256, 0, s>>>(p);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -264,6 +349,7 @@ cudaError_t launch_state_init(int64_t* id_ring, int n_hist, void* v_ring, float*
       id_ring, n_hist, dt == ENGRAM_BF16 ? static_cast<uint16_t*>(v_ring) : nullptr,
       dt == ENGRAM_F32 ? static_cast<float*>(v_ring) : nullptr, g_ring, pos, ring_len, B, H, hc,
       pad_id);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -72,6 +72,7 @@ cudaError_t launch_gather(const GatherParams& p, cudaStream_t s) {
   if (blocks > cap) blocks = cap;
   if (v16) gather_v16_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(p);
   else gather_v4_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(p);
+  count_launch();
   return cudaGetLastError();
 }
 

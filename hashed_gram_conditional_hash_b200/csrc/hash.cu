@@ -135,11 +135,13 @@ cudaError_t launch_hash(const HashParams& p, cudaStream_t s) {
   if (p.B > 0 && p.T > 0) {
     dim3 grid((p.T + 255) / 256, p.B);
     hash_kernel<<<grid, 256, 0, s>>>(p);
+    count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (p.id_ring_out != nullptr && p.n_hist > 0 && p.B > 0) {
     id_ring_kernel<<<(p.B + 127) / 128, 128, 0, s>>>(p);
+    count_launch();
     return cudaGetLastError();
   }
   return cudaSuccess;
@@ -152,6 +154,7 @@ cudaError_t launch_compress(const int64_t* raw, int64_t n, const int64_t* lookup
   int cap = num_sms() * 8;
   if (blocks > cap) blocks = cap;
   compress_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(raw, n, lookup, raw_vocab, out, status);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -127,6 +127,7 @@ cudaError_t launch_proj_simt(const ProjParams& p, cudaStream_t s) {
   dim3 grid((1 + p.hc) * p.H / BN, static_cast<unsigned>((p.M + BM - 1) / BM));
   if (p.dtype == ENGRAM_F32) proj_simt_kernel<float><<<grid, 256, 0, s>>>(p);
   else proj_simt_kernel<uint16_t><<<grid, 256, 0, s>>>(p);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -131,12 +131,22 @@ size_t engram_last_error(char* buf, size_t n);
  * word.  Returns ENGRAM_ERR_TIMEOUT / ENGRAM_ERR_ID_RANGE if those bits are set. */
 engram_status engram_read_status(uint32_t* dev_status, uint32_t* host_bits, engram_stream stream);
 
-/* Test knobs (process-wide).  ENGRAM_DEBUG_FORCE_TIMEOUT makes the next
- * projection launches wait, with a short limit, on a barrier nothing arrives
- * at, so the timeout path runs without a hang.  ENGRAM_DEBUG_FORCE_SIMT selects
- * the CUDA-core projection kernel even where the tensor-core one applies. */
+/* Number of kernels this library has launched in this process (all
+ * devices, all threads).  Lets a caller count the library's launches inside
+ * a timed region. */
+uint64_t engram_launch_count(void);
+
+/* Test and comparison knobs (process-wide).  ENGRAM_DEBUG_FORCE_TIMEOUT makes
+ * the next projection launches wait, with a short limit, on a barrier nothing
+ * arrives at, so the timeout path runs without a hang.  ENGRAM_DEBUG_FORCE_SIMT
+ * selects the CUDA-core projection kernel even where the tensor-core one
+ * applies. */
 #define ENGRAM_DEBUG_FORCE_TIMEOUT 0x1u
 #define ENGRAM_DEBUG_FORCE_SIMT 0x2u
+/* ENGRAM_DEBUG_FUSED_GATHER makes engram_forward feed the table rows straight
+ * into the projection (gathered inside the projection kernel, once per output
+ * tile) instead of gathering e once and projecting it. */
+#define ENGRAM_DEBUG_FUSED_GATHER 0x4u
 void engram_set_debug(uint32_t flags);
 
 /* Which projection engine engram_forward / engram_gate_fuse use for cfg under
@@ -146,6 +156,20 @@ void engram_set_debug(uint32_t flags);
 #define ENGRAM_ENGINE_SIMT 0
 #define ENGRAM_ENGINE_TCGEN05 1
 int32_t engram_projection_engine(const engram_config* cfg);
+
+/* Optional stage timing (process-wide).  When set, engram_forward records
+ * each non-NULL event (a cudaEvent_t owned by the caller) on its stream at
+ * the stage boundaries: before the hash, before the projection, before the
+ * gate, before the conv, after the conv.  NULL disables.  Used by the
+ * benchmark to time the projection kernel inside the full pass. */
+typedef struct {
+  void* before_hash;
+  void* before_projection;
+  void* before_gate;
+  void* before_conv;
+  void* after_conv;
+} engram_stage_events;
+void engram_set_stage_events(const engram_stage_events* events);
 
 /* ---- steps of the pass ----------------------------------------------- */
 

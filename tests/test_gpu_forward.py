@@ -17,9 +17,12 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+ENGINE_FLAGS = {"auto": 0, "simt": L.DEBUG_FORCE_SIMT, "fused": L.DEBUG_FUSED_GATHER,
+                "simt_fused": L.DEBUG_FORCE_SIMT | L.DEBUG_FUSED_GATHER}
+
+
 def _run(p, engine="auto", conv_w=None):
-    if engine == "simt":
-        L.engram_set_debug(L.DEBUG_FORCE_SIMT)
+    L.engram_set_debug(ENGINE_FLAGS[engine])
     try:
         layer = EngramLayer.from_params(p)
         if conv_w is not None:
@@ -39,11 +42,13 @@ SMALL = [
     dict(B=4, T=3, hc_mult=1),
     dict(dtype="f32", B=2, T=50, row_dim=32, hidden=128, hc_mult=3),
     dict(B=2, T=200, heads_per_order=4, hidden=768, hc_mult=2),   # 768 = 3 tiles of 256
+    dict(B=2, T=70, conv_kernel=6, dilation=2),                   # generic tap count
+    dict(B=1, T=150, dilation=9, hc_mult=3),                      # long halo (R = 27)
 ]
 
 
 @pytest.mark.parametrize("kw", SMALL, ids=[str(i) for i in range(len(SMALL))])
-@pytest.mark.parametrize("engine", ["auto", "simt"])
+@pytest.mark.parametrize("engine", ["auto", "simt", "fused", "simt_fused"])
 def test_forward_small_full(kw, engine):
     w = W.small_workload(**kw)
     p = device_params(w)
@@ -88,7 +93,10 @@ def test_forward_engines_agree():
     p = device_params(w)
     a = _run(p, "auto").double()
     b = _run(p, "simt").double()
+    c = _run(p, "fused").double()
     assert (a - b).abs().max().item() <= 2e-2 * b.abs().max().item()
+    # the fused gather feeds the same rows to the same MMA: identical results
+    assert torch.equal(a, c)
 
 
 def test_forward_empty_is_noop():
