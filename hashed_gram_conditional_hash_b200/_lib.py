@@ -93,6 +93,8 @@ def lib() -> C.CDLL:
             "engram_state_init": (C.c_int, [cfg, C.POINTER(EngramState), i32, P]),
             "engram_forward": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P, P,
                                          C.POINTER(EngramState), P, sz, P, P]),
+            "engram_forward_no_alloc": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P,
+                                                  P, C.POINTER(EngramState), P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -273,3 +275,19 @@ def engram_forward(cfg: EngramConfig, weights: EngramWeights, ids: torch.Tensor,
     _check(lib().engram_forward(C.byref(cfg), C.byref(weights), _ptr(ids), B, T, _ptr(hidden),
                                 _ptr(y), C.byref(state) if state is not None else None, _ptr(ws),
                                 ws.numel(), _ptr(dev_status), _stream(stream)))
+
+
+NO_ALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def engram_forward_no_alloc(cfg: EngramConfig, weights: EngramWeights, ids: torch.Tensor,
+                            hidden: torch.Tensor, y: torch.Tensor,
+                            state: Optional[EngramState] = None,
+                            dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """engram_forward in the library's static device scratch (no workspace
+    argument; for callers that cannot allocate device memory)."""
+    B, T = ids.shape
+    _check(lib().engram_forward_no_alloc(C.byref(cfg), C.byref(weights), _ptr(ids), B, T,
+                                         _ptr(hidden), _ptr(y),
+                                         C.byref(state) if state is not None else None,
+                                         _ptr(dev_status), _stream(stream)))

@@ -191,6 +191,14 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 }
 
+engram_status set_error(engram_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 int num_sms() {

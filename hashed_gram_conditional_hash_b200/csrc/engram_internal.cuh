@@ -147,6 +147,9 @@ int num_sms();
 // Count of kernels launched by the library (engram_launch_count).
 void count_launch(int n = 1);
 
+// Sets the calling thread's engram_last_error text and returns st.
+engram_status set_error(engram_status st, const char* fmt, ...);
+
 // ---------------------------------------------------------------- device side
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {

@@ -250,6 +250,36 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wei
                              void* y, const engram_state* state, void* ws, size_t ws_bytes,
                              uint32_t* dev_status, engram_stream stream);
 
+/* ---- the whole pass without caller scratch ----------------------------- */
+
+/* Bytes of the static device scratch engram_forward_no_alloc works in. */
+#define ENGRAM_NO_ALLOC_SCRATCH_BYTES (32u << 20)
+
+/* engram_forward for callers that cannot allocate device memory: a plugin
+ * handed only its input and output buffers by a host framework that owns all
+ * allocation, or a latency-critical loop where cudaMalloc / cudaFree would
+ * synchronise the device.  The paper has no counterpart; this is a property
+ * of the library, not of the method.
+ *
+ * Arguments and results are exactly those of engram_forward minus ws and
+ * ws_bytes: the scratch is a file-scope device array of
+ * ENGRAM_NO_ALLOC_SCRATCH_BYTES (32 MiB) that every GPU which loads the
+ * library holds until the process exits.  A call whose
+ * engram_forward_workspace_size(cfg, B, T) exceeds that size returns
+ * ENGRAM_ERR_INVALID_ARG without launching anything (split the batch).
+ * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  Every call on a device shares the one array and leaves its
+ * contents behind (the pass writes every scratch byte it reads, so nothing
+ * needs clearing); calls that overlap on the GPU, on different streams or
+ * host threads, race on it and give undefined results. */
+engram_status engram_forward_no_alloc(const engram_config* cfg, const engram_weights* weights,
+                                      const int64_t* ids, int32_t B, int32_t T, const void* hidden,
+                                      void* y, const engram_state* state, uint32_t* dev_status,
+                                      engram_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
