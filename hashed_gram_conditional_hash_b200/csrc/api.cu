@@ -129,23 +129,22 @@ StageLayout stage_layout(const engram_config* c, int64_t M, size_t start) {
 
 int64_t rows_ld(int64_t M) { return (M + 127) / 128 * 128; }
 
-// Forward workspace: either (idx [M, nh] int64, e [M, E]) for the gather-then-
-// project path, or the head-major int32 rows [nh, rows_ld(M)] of the fused
-// path, in one shared region; then V, partials and gates.
+// Forward workspace: either e [M, E] for the gather-then-project path, or
+// the head-major int32 rows [nh, rows_ld(M)] of the fused-gather path, in one
+// shared region; then V, partials and gates.
 struct ForwardLayout {
-  size_t idx_off, e_off, rows_off;
+  size_t e_off, rows_off;
   StageLayout st;
 };
 ForwardLayout forward_layout(const engram_config* c, int64_t M) {
   ForwardLayout L;
   const int nh = c->n_orders * c->heads_per_order;
   const size_t es = c->dtype == ENGRAM_F32 ? 4 : 2;
-  L.idx_off = 0;
-  L.e_off = align256(static_cast<size_t>(M) * nh * sizeof(int64_t));
-  const size_t split_end = align256(L.e_off + static_cast<size_t>(M) * nh * c->row_dim * es);
+  L.e_off = 0;
   L.rows_off = 0;
+  const size_t e_end = align256(static_cast<size_t>(M) * nh * c->row_dim * es);
   const size_t rows_end = align256(static_cast<size_t>(nh) * rows_ld(M) * sizeof(int32_t));
-  L.st = stage_layout(c, M, split_end > rows_end ? split_end : rows_end);
+  L.st = stage_layout(c, M, e_end > rows_end ? e_end : rows_end);
   return L;
 }
 
@@ -161,8 +160,10 @@ engram_status run_projection(const engram_config* c, ProjParams* pp, cudaStream_
   pp->n_tiles = c->hidden / (tc ? kTcTileN : kSimtTileN);
   pp->debug = g_debug.load();
   record(g_events.before_projection, s);
-  engram_status st = tc ? cuda_check(launch_proj_tc(*pp, s), "projection (tcgen05)")
-                        : cuda_check(launch_proj_simt(*pp, s), "projection (SIMT)");
+  const bool pairs = tc && pp->rows == nullptr && (pp->debug & ENGRAM_DEBUG_TC_SINGLE_CTA) == 0;
+  engram_status st = pairs ? cuda_check(launch_proj_tc2(*pp, s), "projection (tcgen05, CTA pairs)")
+                   : tc    ? cuda_check(launch_proj_tc(*pp, s), "projection (tcgen05)")
+                           : cuda_check(launch_proj_simt(*pp, s), "projection (SIMT)");
   record(g_events.before_gate, s);
   return st;
 }
@@ -491,11 +492,13 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   char* w = static_cast<char*>(ws);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  // a1-a3: ids -> hash indices (or absolute table rows for the fused path)
-  const bool fused = (g_debug.load() & ENGRAM_DEBUG_FUSED_GATHER) != 0;
+  // a1-a4: ids -> e (hash and gather in one kernel), or -> absolute table
+  // rows for the fused-gather path (rows with a width that is not a multiple
+  // of 16 bytes also take that path: the projection gathers them itself)
+  const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
+  const bool fused = (g_debug.load() & ENGRAM_DEBUG_FUSED_GATHER) != 0 || (row_bytes % 16) != 0;
   const int64_t ld = rows_ld(M);
   int32_t* rows = reinterpret_cast<int32_t*>(w + L.rows_off);
-  int64_t* idx = reinterpret_cast<int64_t*>(w + L.idx_off);
   void* e = w + L.e_off;
   hp.ids = ids;
   hp.lookup = wts->lookup;
@@ -503,31 +506,23 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   hp.history = state != nullptr ? state->id_ring : nullptr;
   hp.id_ring_out = state != nullptr ? state->id_ring : nullptr;
   hp.rows_out = fused ? rows : nullptr;
-  hp.idx_out = fused ? nullptr : idx;
+  hp.idx_out = nullptr;
   hp.ld_rows = ld;
   hp.status = dev_status;
   hp.B = B;
   hp.T = T;
   record(g_events.before_hash, s);
-  st = cuda_check(launch_hash(hp, s), "hash");
-  if (st != ENGRAM_OK) return st;
-
-  // a4: e = the gathered rows, once (unless fused into the projection)
-  if (!fused) {
-    GatherParams gp;
-    memset(&gp, 0, sizeof gp);
-    gp.table = wts->table;
-    gp.idx = idx;
-    gp.e = e;
-    gp.status = dev_status;
-    gp.M = M;
-    gp.total_rows = wts->total_rows;
-    gp.nh = hp.nh;
-    gp.row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
-    for (int h = 0; h < hp.nh; ++h) gp.row_off[h] = hp.row_off[h];
-    st = cuda_check(launch_gather(gp, s), "gather");
-    if (st != ENGRAM_OK) return st;
+  if (fused) {
+    st = cuda_check(launch_hash(hp, s), "hash");
+  } else {
+    HashGatherParams hg;
+    hg.h = hp;
+    hg.table = wts->table;
+    hg.e = e;
+    hg.row_bytes = row_bytes;
+    st = cuda_check(launch_hash_gather(hg, s), "hash+gather");
   }
+  if (st != ENGRAM_OK) return st;
 
   // a5-a7: projection, score partials, gates
   ProjParams pp;

@@ -40,6 +40,16 @@ cudaError_t launch_hash(const HashParams& p, cudaStream_t s);
 cudaError_t launch_compress(const int64_t* raw, int64_t n, const int64_t* lookup,
                             int64_t raw_vocab, int64_t* out, uint32_t* status, cudaStream_t s);
 
+// Hash and gather in one pass (a1-a4 inside engram_forward): e[m, h*Dh..] =
+// table[row_off[h] + hash(m, h)], rows of row_bytes (a multiple of 16).
+struct HashGatherParams {
+  HashParams h;             // ids, lookup, history, multipliers, primes, row offsets
+  const void* table;
+  void* e;                  // [B*T, nh*Dh]
+  int32_t row_bytes;
+};
+cudaError_t launch_hash_gather(const HashGatherParams& p, cudaStream_t s);
+
 // Row gather (a4): e[m, h*Dh + c] = table[off[h] + idx[m, h], c].
 struct GatherParams {
   const void* table;
@@ -84,6 +94,8 @@ constexpr int kTcTileN = 128;
 bool tc_projection_supported(int Dh, int H, engram_dtype dt);
 cudaError_t launch_proj_simt(const ProjParams& p, cudaStream_t s);
 cudaError_t launch_proj_tc(const ProjParams& p, cudaStream_t s);
+// Dense A only, on CTA pairs (2-SM MMA).
+cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s);
 
 // Gate finalisation (a6 reduction + a7): g[m, h] from the partials.
 struct GateParams {

@@ -82,6 +82,38 @@ template <> struct Vec8<float> {
   }
 };
 
+// Eight channels kept in their stored form (packed bf16 or floats).
+template <typename T> struct Raw8;
+template <> struct Raw8<uint16_t> {
+  using type = uint4;
+  static __device__ __forceinline__ uint4 load(const uint16_t* p) {
+    return __ldg(reinterpret_cast<const uint4*>(p));
+  }
+  static __device__ __forceinline__ uint4 zero() { return make_uint4(0, 0, 0, 0); }
+  static __device__ __forceinline__ void unpack(const uint4& w, float (&v)[8]) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(u[i] << 16);
+      v[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+  }
+};
+struct F8 { float4 a, b; };
+template <> struct Raw8<float> {
+  using type = F8;
+  static __device__ __forceinline__ F8 load(const float* p) {
+    return F8{__ldg(reinterpret_cast<const float4*>(p)), __ldg(reinterpret_cast<const float4*>(p) + 1)};
+  }
+  static __device__ __forceinline__ F8 zero() {
+    return F8{make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+  }
+  static __device__ __forceinline__ void unpack(const F8& w, float (&v)[8]) {
+    v[0] = w.a.x; v[1] = w.a.y; v[2] = w.a.z; v[3] = w.a.w;
+    v[4] = w.b.x; v[5] = w.b.y; v[6] = w.b.z; v[7] = w.b.w;
+  }
+};
+
 constexpr int kConvThreads = 256;
 
 // Conv taps of 8 consecutive channels: w[j][i] = row[j*K + i] (8K contiguous
@@ -193,6 +225,86 @@ __global__ void __launch_bounds__(kConvThreads) gated_conv_kernel(const __grid_c
   }
 }
 
+// Run form for the pages' kernel of K = 4 taps.  The taps of position t are
+// t - 3 dil, t - 2 dil, t - dil, t: all in t's residue class mod dil.  A
+// thread owns 8 channels of one branch along a run of RUN consecutive
+// positions of one residue class: it issues every load of the run at once
+// (RUN + 3 V rows of 16 bytes, kept packed, and their gates), then produces
+// RUN outputs from registers with that branch's taps.  Each V row is read by
+// a handful of threads through L1/L2; DRAM sees it about once.
+template <typename T, int RUN>
+__global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_constant__ ConvParams p) {
+  constexpr int K = 4;
+  constexpr int NW = RUN + K - 1;                 // rows in the window of a run
+  const int cgs = p.H >> 3;
+  const int64_t gid = blockIdx.x * static_cast<int64_t>(kConvThreads) + threadIdx.x;
+  const int runs_per_class = (p.T + p.dil * RUN - 1) / (p.dil * RUN);
+  // thread order: (b, residue class, run, branch, channel group), channel group fastest
+  const int64_t per_run = static_cast<int64_t>(p.hc) * cgs;
+  const int64_t per_b = static_cast<int64_t>(p.dil) * runs_per_class * per_run;
+  if (gid >= per_b * p.B) return;
+  const int b = static_cast<int>(gid / per_b);
+  int64_t rem = gid - b * per_b;
+  const int cls = static_cast<int>(rem / (static_cast<int64_t>(runs_per_class) * per_run));
+  rem -= static_cast<int64_t>(cls) * runs_per_class * per_run;
+  const int jr = static_cast<int>(rem / per_run);
+  rem -= static_cast<int64_t>(jr) * per_run;
+  const int h = static_cast<int>(rem / cgs);
+  const int c = static_cast<int>(rem - static_cast<int64_t>(h) * cgs) * 8;
+  const int t_first = cls + p.dil * (jr * RUN);   // first output position of the run
+  if (t_first >= p.T) return;
+  const T* V = static_cast<const T*>(p.V);
+  const T* vr = static_cast<const T*>(p.v_ring);
+  T* Y = static_cast<T*>(p.Y);
+  const int64_t seq = static_cast<int64_t>(b) * p.T;
+  const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) : 0;
+
+  // window row k is position t_first + (k - 3) * dil
+  typename Raw8<T>::type vraw[NW];
+  float gw[NW];
+#pragma unroll
+  for (int k = 0; k < NW; ++k) {
+    const int tp = t_first + (k - (K - 1)) * p.dil;
+    const float* gsrc = nullptr;
+    const T* vsrc = nullptr;
+    if (tp >= 0 && tp < p.T) {
+      gsrc = p.g + (seq + tp) * p.hc + h;
+      vsrc = V + (seq + tp) * p.H + c;
+    } else if (tp < 0 && vr != nullptr && P + tp >= 0) {
+      const int64_t rb = static_cast<int64_t>(b) * p.ring_len + (P + tp) % p.ring_len;
+      gsrc = p.g_ring + rb * p.hc + h;
+      vsrc = vr + rb * p.H + c;
+    }
+    if (vsrc != nullptr) {
+      vraw[k] = Raw8<T>::load(vsrc);
+      gw[k] = __ldg(gsrc);
+    } else {
+      vraw[k] = Raw8<T>::zero();
+      gw[k] = 0.f;
+    }
+  }
+  float w[8][K];
+  load_taps<T, K>(static_cast<const T*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, K, w);
+#pragma unroll
+  for (int q = 0; q < RUN; ++q) {
+    const int t = t_first + q * p.dil;
+    if (t < p.T) {
+      float v[K][8];
+#pragma unroll
+      for (int i = 0; i < K; ++i) Raw8<T>::unpack(vraw[q + i], v[i]);
+      float acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float a = gw[q + K - 1] * v[K - 1][j];                 // U(t)
+#pragma unroll
+        for (int i = 0; i < K; ++i) a = fmaf(w[j][i], gw[q + i] * v[i][j], a);
+        acc[j] = a;
+      }
+      Vec8<T>::store(Y + ((seq + t) * p.hc + h) * p.H + c, acc);
+    }
+  }
+}
+
 // -------------------------------------------------------------- standalone conv
 template <typename T>
 __global__ void short_conv_kernel(const __grid_constant__ ShortConvParams p) {
@@ -294,7 +406,16 @@ cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
   const int64_t blocks = (threads + kConvThreads - 1) / kConvThreads;
   if (blocks > INT32_MAX) return cudaErrorInvalidValue;
   const unsigned nb = static_cast<unsigned>(blocks);
-  if (p.K <= 4 && p.hc <= 4) {  // the pages' shape: kernel 4, up to 4 branches
+  constexpr int kRun = 8;
+  if (p.K == 4 && p.conv_w != nullptr && p.T >= 2 * kRun * p.dil) {
+    // run form along each residue class mod dil (the pages' kernel of 4 taps)
+    const int64_t rpc = (p.T + static_cast<int64_t>(p.dil) * kRun - 1) / (static_cast<int64_t>(p.dil) * kRun);
+    const int64_t nthreads = static_cast<int64_t>(p.B) * p.dil * rpc * p.hc * (p.H / 8);
+    const int64_t rb = (nthreads + kConvThreads - 1) / kConvThreads;
+    if (rb > INT32_MAX) return cudaErrorInvalidValue;
+    if (p.dtype == ENGRAM_F32) conv_run_kernel<float, kRun><<<static_cast<unsigned>(rb), kConvThreads, 0, s>>>(p);
+    else conv_run_kernel<uint16_t, kRun><<<static_cast<unsigned>(rb), kConvThreads, 0, s>>>(p);
+  } else if (p.K <= 4 && p.hc <= 4) {  // up to 4 taps and 4 branches
     if (p.dtype == ENGRAM_F32) gated_conv_kernel<float, 4, 4><<<nb, kConvThreads, 0, s>>>(p);
     else gated_conv_kernel<uint16_t, 4, 4><<<nb, kConvThreads, 0, s>>>(p);
   } else {

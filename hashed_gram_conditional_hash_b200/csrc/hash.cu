@@ -114,6 +114,71 @@ __global__ void id_ring_kernel(const __grid_constant__ HashParams p) {
   }
 }
 
+// Id at position t of sequence b (pad / history before the start), compressed
+// and range-checked.
+__device__ __forceinline__ uint64_t token_at(const HashParams& p, int b, int t) {
+  if (t >= 0) return static_cast<uint64_t>(load_id(p, __ldg(p.ids + static_cast<int64_t>(b) * p.T + t)));
+  if (p.history != nullptr && -t <= p.n_hist) {
+    int64_t hv = __ldg(p.history + static_cast<int64_t>(b) * p.n_hist + p.n_hist + t);
+    if (hv < 0 || hv >= p.vocab) {
+      set_status(p.status, ENGRAM_STATUS_ID_RANGE);
+      hv = p.pad_id;
+    }
+    return static_cast<uint64_t>(hv);
+  }
+  return static_cast<uint64_t>(p.pad_id);
+}
+
+// One warp produces 32 consecutive rows of e (row q = m*nh + h): lane l
+// hashes row q0 + l (its order's window read through L1, xor of products,
+// Barrett reduction by its head's prime), then the warp copies the 32 table
+// rows with every 16-byte load issued before the stores.
+__global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant__ HashGatherParams g) {
+  const HashParams& p = g.h;
+  const int lane = threadIdx.x & 31;
+  const int64_t M = static_cast<int64_t>(p.B) * p.T;
+  const int64_t total = M * p.nh;
+  const int64_t q0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) - lane;
+  if (q0 >= total) return;
+  const int64_t q = q0 + lane;
+  int64_t row = 0;
+  if (q < total) {
+    const int64_t m = q / p.nh;
+    const int h = static_cast<int>(q - m * p.nh);
+    const int o = h / p.J;
+    const int b = static_cast<int>(m / p.T);
+    const int t = static_cast<int>(m - static_cast<int64_t>(b) * p.T);
+    const int n = p.orders[o];
+    uint64_t mix = token_at(p, b, t) * p.mult[0];
+#pragma unroll
+    for (int k = 1; k < ENGRAM_MAX_NGRAM; ++k)
+      if (k < n) mix ^= token_at(p, b, t - k) * p.mult[k];
+    row = p.row_off[h] + static_cast<int64_t>(barrett_mod(mix, p.prime[h], p.barrett[h]));
+  }
+  const int chunks = g.row_bytes >> 4;          // 16-byte chunks per row
+  const int per = 32 * chunks;                   // chunks of this warp's 32 rows
+  const char* tab = static_cast<const char*>(g.table);
+  int4* out = static_cast<int4*>(g.e) + q0 * chunks;
+  constexpr int kBatch = 8;
+  for (int base = 0; base < per; base += 32 * kBatch) {
+    int4 v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * 32 + lane;
+      const int r = i / chunks;
+      const int64_t src = __shfl_sync(0xffffffffu, row, r & 31);
+      if (i < per && q0 + r < total)
+        v[u] = __ldg(reinterpret_cast<const int4*>(tab + src * g.row_bytes) + (i - r * chunks));
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * 32 + lane;
+      const int r = i / chunks;
+      if (i < per && q0 + r < total) out[i] = v[u];
+    }
+  }
+}
+
 __global__ void compress_kernel(const int64_t* __restrict__ raw, int64_t n,
                                 const int64_t* __restrict__ lookup, int64_t raw_vocab,
                                 int64_t* __restrict__ out, uint32_t* status) {
@@ -135,6 +200,25 @@ cudaError_t launch_hash(const HashParams& p, cudaStream_t s) {
   if (p.B > 0 && p.T > 0) {
     dim3 grid((p.T + 255) / 256, p.B);
     hash_kernel<<<grid, 256, 0, s>>>(p);
+    count_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (p.id_ring_out != nullptr && p.n_hist > 0 && p.B > 0) {
+    id_ring_kernel<<<(p.B + 127) / 128, 128, 0, s>>>(p);
+    count_launch();
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_hash_gather(const HashGatherParams& g, cudaStream_t s) {
+  const HashParams& p = g.h;
+  const int64_t total = static_cast<int64_t>(p.B) * p.T * p.nh;
+  if (total > 0) {
+    const int64_t blocks = (total + 255) / 256;
+    if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+    hash_gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(g);
     count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -147,6 +147,9 @@ uint64_t engram_launch_count(void);
  * into the projection (gathered inside the projection kernel, once per output
  * tile) instead of gathering e once and projecting it. */
 #define ENGRAM_DEBUG_FUSED_GATHER 0x4u
+/* ENGRAM_DEBUG_TC_SINGLE_CTA runs the dense tensor-core projection on single
+ * CTAs (128 x 256 tiles) instead of CTA pairs (256 x 256 tiles, 2-SM MMA). */
+#define ENGRAM_DEBUG_TC_SINGLE_CTA 0x8u
 void engram_set_debug(uint32_t flags);
 
 /* Which projection engine engram_forward / engram_gate_fuse use for cfg under

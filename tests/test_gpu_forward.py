@@ -18,7 +18,8 @@ DEV = "cuda"
 
 
 ENGINE_FLAGS = {"auto": 0, "simt": L.DEBUG_FORCE_SIMT, "fused": L.DEBUG_FUSED_GATHER,
-                "simt_fused": L.DEBUG_FORCE_SIMT | L.DEBUG_FUSED_GATHER}
+                "simt_fused": L.DEBUG_FORCE_SIMT | L.DEBUG_FUSED_GATHER,
+                "single_cta": L.DEBUG_TC_SINGLE_CTA}
 
 
 def _run(p, engine="auto", conv_w=None):
@@ -44,11 +45,13 @@ SMALL = [
     dict(B=2, T=200, heads_per_order=4, hidden=768, hc_mult=2),   # 768 = 3 tiles of 256
     dict(B=2, T=70, conv_kernel=6, dilation=2),                   # generic tap count
     dict(B=1, T=150, dilation=9, hc_mult=3),                      # long halo (R = 27)
+    dict(B=2, T=45, row_dim=20),                                  # 40-byte rows
+    dict(B=2, T=90, hc_mult=6, hidden=128),                       # more than 4 branches
 ]
 
 
 @pytest.mark.parametrize("kw", SMALL, ids=[str(i) for i in range(len(SMALL))])
-@pytest.mark.parametrize("engine", ["auto", "simt", "fused", "simt_fused"])
+@pytest.mark.parametrize("engine", ["auto", "simt", "fused", "simt_fused", "single_cta"])
 def test_forward_small_full(kw, engine):
     w = W.small_workload(**kw)
     p = device_params(w)
@@ -68,10 +71,11 @@ def test_forward_tiny_f32_full():
 
 @pytest.mark.parametrize("name,n_random", [("model_bf16", 48), ("large_table_bf16", 24),
                                            ("hbm_table_bf16", 16)])
-def test_forward_full_size_sampled(name, n_random):
+@pytest.mark.parametrize("engine", ["auto", "single_cta"])
+def test_forward_full_size_sampled(name, n_random, engine):
     w = W.CONFIGS[name]
     p = device_params(w)
-    y = _run(p)
+    y = _run(p, engine)
     pos = sample_positions(w.B, w.T, w.dil, n_random, seed=11)
     Yref, s, g, _ = oracle_at(p, pos)
     got = torch.stack([y[b, t] for b, t in pos]).double().cpu().numpy()
@@ -94,9 +98,11 @@ def test_forward_engines_agree():
     a = _run(p, "auto").double()
     b = _run(p, "simt").double()
     c = _run(p, "fused").double()
+    d = _run(p, "single_cta").double()
     assert (a - b).abs().max().item() <= 2e-2 * b.abs().max().item()
-    # the fused gather feeds the same rows to the same MMA: identical results
-    assert torch.equal(a, c)
+    # the fused gather feeds the same rows to the single-CTA MMA: identical results
+    assert torch.equal(c, d)
+    assert (a - d).abs().max().item() <= 1e-2 * d.abs().max().item()
 
 
 def test_forward_empty_is_noop():
