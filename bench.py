@@ -113,9 +113,12 @@ def oracle_sample(w, tokens: int, nthreads: int):
     from ids, host cores).  Returns (n, run) where run() -> seconds."""
     from hashed_gram_conditional_hash_b200 import workloads as W
     from oracle import engram_oracle as O
-    n = max(1, min(tokens, w.seq_len))
+    n = max(1, min(tokens, w.B * w.seq_len))
     if W.gen_device_for(w, "cuda") == "cpu":
-        wp = w.replace(B=1, T=n, decode_calls=0)
+        # whole sequences of the workload's length (the last one cut to fit)
+        T = min(n, w.seq_len)
+        wp = w.replace(B=(n + T - 1) // T, T=T, decode_calls=0)
+        n = wp.B * wp.T
         p = W.make_params(wp, "cpu")
         x = p.ids.numpy()
         if p.lookup is not None:
@@ -133,6 +136,7 @@ def oracle_sample(w, tokens: int, nthreads: int):
     # tables drawn on the device: the oracle receives the rows it needs
     p = W.make_params(w, "cuda")
     dev = p.table.device
+    n = min(n, w.seq_len)
     pos = [(0, t) for t in range(n)]
     if w.decode_calls:
         hid = lambda b, t: p.hidden[torch.from_numpy(t).to(dev), torch.from_numpy(b).to(dev)].cpu()
@@ -163,11 +167,27 @@ def cpu_baseline(w, budget_s: float):
     n, run = oracle_sample(w, oracle_tokens_for(w, budget_s, nthreads), nthreads)
     dt = run()
     return {"value": n / dt, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
-            "sample": "first %d positions of sequence 0 of workload %s (same shapes and "
-                      "distributions), whole pass from ids, float64, %.1f s" % (n, w.name, dt)}
+            "sample": "%d positions (whole sequences) of a workload with the shapes and "
+                      "distributions of %s, whole pass from ids, float64, %.1f s" % (n, w.name, dt)}
 
 
 # ---------------------------------------------------------------- GPU arm
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    record (profiles/dram_traffic.json), only if the kernel's source file is
+    unchanged since that capture; else None."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f)["%s@%s" % (kernel, workload)]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != rec["source_sha1"]:
+                return None
+        return rec["dram_read_bytes"] + rec["dram_write_bytes"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def algorithmic(w):
     """Per-token algorithmic bytes / flops of each stage (see the design notes)."""
     es = w.elem_bytes
@@ -186,10 +206,14 @@ def run_ours(args, rank, world, device):
     from hashed_gram_conditional_hash_b200 import workloads as W
 
     w = W.CONFIGS[args.config]
+    if w.decode_calls and args.decode_calls:
+        w = w.replace(decode_calls=args.decode_calls)
     peaks, peak_kind = load_peaks()
     p = W.make_params(w, device)
     layer = EngramLayer.from_params(p)
     engine = "tcgen05" if L.engram_projection_engine(layer.cfg) == L.ENGINE_TCGEN05 else "simt"
+    # the dense tensor-core projection runs on CTA pairs
+    kname = "proj_tc2_kernel" if engine == "tcgen05" else "proj_simt_kernel"
     stream = torch.cuda.current_stream()
     decode = bool(w.decode_calls)
     if decode:
@@ -289,10 +313,10 @@ def run_ours(args, rank, world, device):
                    "dilation": w.dil, "table_gb": round(W.table_bytes(w) / 1e9, 3),
                    "l2": "flushed (256 MB write) between timed steps",
                    "parallelism": "replicas x%d" % world, "projection_engine": engine},
-        "roofline": {"bound": "tensor", "kernel": "proj_tc_kernel" if engine == "tcgen05" else "proj_simt_kernel",
+        "roofline": {"bound": "tensor", "kernel": kname,
                      "achieved": proj_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": proj_tflops / tc_peak, "peak_kind": "%s bf16 burst" % peak_kind,
-                     "traffic": None,
+                     "traffic": kernel_traffic(kname, w.name),
                      "flops_per_launch": a["proj_flops"] * tokens_step},
         "stages": stages,
         "clocks": clk,
@@ -364,8 +388,8 @@ def run_reference(args):
     for _ in range(args.steps):
         tot += run()
     rate = n * args.steps / tot
-    sample = ("per step: first %d positions of sequence 0 of workload %s (same shapes and "
-              "distributions), whole pass from ids, float64 oracle" % (n, w.name))
+    sample = ("per step: %d positions (whole sequences) of a workload with the shapes and "
+              "distributions of %s, whole pass from ids, float64 oracle" % (n, w.name))
     return {
         "impl": "reference",
         "metric": "Engram forward tokens/s on 1xB200 (engram_forward); % of HBM and bf16 tensor roofline",
@@ -390,6 +414,8 @@ def main():
     ap.add_argument("--ref-step-s", type=float, default=3.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--decode-calls", type=int, default=0,
+                    help="decode workload: number of distinct calls drawn (default: all 256)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

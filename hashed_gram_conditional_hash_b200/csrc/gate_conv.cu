@@ -61,12 +61,8 @@ template <> struct Vec8<uint16_t> {
     }
   }
   static __device__ __forceinline__ void store(uint16_t* p, const float (&v)[8]) {
-    uint4 w;
-    w.x = static_cast<uint32_t>(f32_to_bf16(v[0])) | (static_cast<uint32_t>(f32_to_bf16(v[1])) << 16);
-    w.y = static_cast<uint32_t>(f32_to_bf16(v[2])) | (static_cast<uint32_t>(f32_to_bf16(v[3])) << 16);
-    w.z = static_cast<uint32_t>(f32_to_bf16(v[4])) | (static_cast<uint32_t>(f32_to_bf16(v[5])) << 16);
-    w.w = static_cast<uint32_t>(f32_to_bf16(v[6])) | (static_cast<uint32_t>(f32_to_bf16(v[7])) << 16);
-    *reinterpret_cast<uint4*>(p) = w;
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
   }
 };
 template <> struct Vec8<float> {
@@ -236,21 +232,24 @@ template <typename T, int RUN>
 __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_constant__ ConvParams p) {
   constexpr int K = 4;
   constexpr int NW = RUN + K - 1;                 // rows in the window of a run
+  // thread order: (b, residue class, run, branch, channel group), channel
+  // group fastest; the launcher keeps the thread count below 2^31, so the
+  // decode is 32-bit
   const int cgs = p.H >> 3;
-  const int64_t gid = blockIdx.x * static_cast<int64_t>(kConvThreads) + threadIdx.x;
+  const int gid = static_cast<int>(blockIdx.x) * kConvThreads + static_cast<int>(threadIdx.x);
   const int runs_per_class = (p.T + p.dil * RUN - 1) / (p.dil * RUN);
-  // thread order: (b, residue class, run, branch, channel group), channel group fastest
-  const int64_t per_run = static_cast<int64_t>(p.hc) * cgs;
-  const int64_t per_b = static_cast<int64_t>(p.dil) * runs_per_class * per_run;
+  const int per_run = p.hc * cgs;
+  const int per_cls = runs_per_class * per_run;
+  const int per_b = p.dil * per_cls;
   if (gid >= per_b * p.B) return;
-  const int b = static_cast<int>(gid / per_b);
-  int64_t rem = gid - b * per_b;
-  const int cls = static_cast<int>(rem / (static_cast<int64_t>(runs_per_class) * per_run));
-  rem -= static_cast<int64_t>(cls) * runs_per_class * per_run;
-  const int jr = static_cast<int>(rem / per_run);
-  rem -= static_cast<int64_t>(jr) * per_run;
-  const int h = static_cast<int>(rem / cgs);
-  const int c = static_cast<int>(rem - static_cast<int64_t>(h) * cgs) * 8;
+  const int b = gid / per_b;
+  int rem = gid - b * per_b;
+  const int cls = rem / per_cls;
+  rem -= cls * per_cls;
+  const int jr = rem / per_run;
+  rem -= jr * per_run;
+  const int h = rem / cgs;
+  const int c = (rem - h * cgs) * 8;
   const int t_first = cls + p.dil * (jr * RUN);   // first output position of the run
   if (t_first >= p.T) return;
   const T* V = static_cast<const T*>(p.V);
@@ -285,19 +284,33 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
   }
   float w[8][K];
   load_taps<T, K>(static_cast<const T*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, K, w);
+  // sliding window of U = g * V: each row is unpacked and scaled once
+  float u[K][8];
+#pragma unroll
+  for (int k = 0; k < K - 1; ++k) {
+    float v[8];
+    Raw8<T>::unpack(vraw[k], v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) u[k + 1][j] = gw[k] * v[j];
+  }
 #pragma unroll
   for (int q = 0; q < RUN; ++q) {
+#pragma unroll
+    for (int i = 0; i < K - 1; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) u[i][j] = u[i + 1][j];
+    float v[8];
+    Raw8<T>::unpack(vraw[q + K - 1], v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) u[K - 1][j] = gw[q + K - 1] * v[j];    // U(t)
     const int t = t_first + q * p.dil;
     if (t < p.T) {
-      float v[K][8];
-#pragma unroll
-      for (int i = 0; i < K; ++i) Raw8<T>::unpack(vraw[q + i], v[i]);
       float acc[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        float a = gw[q + K - 1] * v[K - 1][j];                 // U(t)
+        float a = u[K - 1][j];
 #pragma unroll
-        for (int i = 0; i < K; ++i) a = fmaf(w[j][i], gw[q + i] * v[i][j], a);
+        for (int i = 0; i < K; ++i) a = fmaf(w[j][i], u[i][j], a);
         acc[j] = a;
       }
       Vec8<T>::store(Y + ((seq + t) * p.hc + h) * p.H + c, acc);
@@ -408,13 +421,17 @@ cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
   const unsigned nb = static_cast<unsigned>(blocks);
   constexpr int kRun = 8;
   if (p.K == 4 && p.conv_w != nullptr && p.T >= 2 * kRun * p.dil) {
-    // run form along each residue class mod dil (the pages' kernel of 4 taps)
-    const int64_t rpc = (p.T + static_cast<int64_t>(p.dil) * kRun - 1) / (static_cast<int64_t>(p.dil) * kRun);
+    // run form along each residue class mod dil (the pages' kernel of 4 taps);
+    // short chunks (decode) take the flat form below, which shares the taps'
+    // loads across the branches
+    const int run = kRun;
+    const int64_t rpc = (p.T + static_cast<int64_t>(p.dil) * run - 1) / (static_cast<int64_t>(p.dil) * run);
     const int64_t nthreads = static_cast<int64_t>(p.B) * p.dil * rpc * p.hc * (p.H / 8);
     const int64_t rb = (nthreads + kConvThreads - 1) / kConvThreads;
-    if (rb > INT32_MAX) return cudaErrorInvalidValue;
-    if (p.dtype == ENGRAM_F32) conv_run_kernel<float, kRun><<<static_cast<unsigned>(rb), kConvThreads, 0, s>>>(p);
-    else conv_run_kernel<uint16_t, kRun><<<static_cast<unsigned>(rb), kConvThreads, 0, s>>>(p);
+    if (rb * kConvThreads > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit thread ids
+    const unsigned g = static_cast<unsigned>(rb);
+    if (p.dtype == ENGRAM_F32) conv_run_kernel<float, kRun><<<g, kConvThreads, 0, s>>>(p);
+    else conv_run_kernel<uint16_t, kRun><<<g, kConvThreads, 0, s>>>(p);
   } else if (p.K <= 4 && p.hc <= 4) {  // up to 4 taps and 4 branches
     if (p.dtype == ENGRAM_F32) gated_conv_kernel<float, 4, 4><<<nb, kConvThreads, 0, s>>>(p);
     else gated_conv_kernel<uint16_t, 4, 4><<<nb, kConvThreads, 0, s>>>(p);

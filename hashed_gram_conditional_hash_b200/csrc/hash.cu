@@ -136,18 +136,18 @@ __device__ __forceinline__ uint64_t token_at(const HashParams& p, int b, int t) 
 __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant__ HashGatherParams g) {
   const HashParams& p = g.h;
   const int lane = threadIdx.x & 31;
-  const int64_t M = static_cast<int64_t>(p.B) * p.T;
-  const int64_t total = M * p.nh;
-  const int64_t q0 = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) - lane;
+  // rows of e (B*T*nh) stay below 2^31 (checked by the launcher): 32-bit math
+  const int total = p.B * p.T * p.nh;
+  const int q0 = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x) - lane;
   if (q0 >= total) return;
-  const int64_t q = q0 + lane;
+  const int q = q0 + lane;
   int64_t row = 0;
   if (q < total) {
-    const int64_t m = q / p.nh;
-    const int h = static_cast<int>(q - m * p.nh);
+    const int m = q / p.nh;
+    const int h = q - m * p.nh;
     const int o = h / p.J;
-    const int b = static_cast<int>(m / p.T);
-    const int t = static_cast<int>(m - static_cast<int64_t>(b) * p.T);
+    const int b = m / p.T;
+    const int t = m - b * p.T;
     const int n = p.orders[o];
     uint64_t mix = token_at(p, b, t) * p.mult[0];
 #pragma unroll
@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant_
   const int chunks = g.row_bytes >> 4;          // 16-byte chunks per row
   const int per = 32 * chunks;                   // chunks of this warp's 32 rows
   const char* tab = static_cast<const char*>(g.table);
-  int4* out = static_cast<int4*>(g.e) + q0 * chunks;
+  int4* out = static_cast<int4*>(g.e) + static_cast<int64_t>(q0) * chunks;
   constexpr int kBatch = 8;
   for (int base = 0; base < per; base += 32 * kBatch) {
     int4 v[kBatch];
@@ -217,7 +217,7 @@ cudaError_t launch_hash_gather(const HashGatherParams& g, cudaStream_t s) {
   const int64_t total = static_cast<int64_t>(p.B) * p.T * p.nh;
   if (total > 0) {
     const int64_t blocks = (total + 255) / 256;
-    if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+    if (blocks * 256 > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit row ids in the kernel
     hash_gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(g);
     count_launch();
     cudaError_t e = cudaGetLastError();

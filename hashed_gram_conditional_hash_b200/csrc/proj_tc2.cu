@@ -24,7 +24,15 @@
 //              128 columns per thread): V -> bf16, or the score partials
 //              against the hidden-state slice (loaded before the wait); the
 //              accumulator is released on the leader's barrier
-// Accumulators are double-buffered (2 x 256 fp32 columns); 6 stages of 32 KB.
+// Accumulators are double-buffered (2 x 256 fp32 columns).
+//
+// TMA delivers a fixed number of boxes per SM per second (measured on B200:
+// 16 KB boxes stream at ~56 GB/s per SM, 32 KB boxes at ~112 GB/s, at any
+// pipeline depth), so each load moves KC = 2 K-blocks at once through a 3-D
+// view of the operand ({64 columns, rows, 64-column chunks}, box {64, 128, 2}):
+// the box lands as two consecutive 128-byte-swizzled 128 x 64 tiles, exactly
+// the UMMA layout of two K-blocks.  Stages hold KC K-blocks (3 stages of 64 KB
+// for KC = 2; 6 stages of 32 KB for KC = 1, used when the head count is odd).
 // Every wait is bounded; an abort raises the flag in both CTAs; no multicast
 // loads are used anywhere (only the commit arrives on both CTAs' barriers).
 #include <cuda.h>
@@ -42,16 +50,16 @@ constexpr int kBM = 128;                    // token rows per CTA (pair: 256)
 constexpr int kBN = 256;                    // output columns per pair tile
 constexpr int kBNh = kBN / 2;               // weight rows per CTA
 constexpr int kBK = 64;
-constexpr int kStages = 6;
-constexpr int kABytes = kBM * kBK * 2;      // 16 KB
-constexpr int kBBytes = kBNh * kBK * 2;     // 16 KB
-constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kStageMem = 192 * 1024;       // operand ring per CTA
+constexpr int kATile = kBM * kBK * 2;       // 16 KB: one K-block of A
+constexpr int kBTile = kBNh * kBK * 2;      // 16 KB: one K-block of this CTA's B half
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kEpiCols = kBN / 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_bf16(2 * kBM, kBN);
-constexpr int kNumBars = 2 * kStages + 2 + 2 + 2;  // full, empty, tfull, tempty, never, drain
+constexpr int kMaxStages = 6;
+constexpr int kNumBars = 2 * kMaxStages + 2 + 2 + 2;  // full, empty, tfull, tempty, never, drain
 
 struct Tc2Params {
   ProjParams p;
@@ -61,9 +69,15 @@ struct Tc2Params {
   int32_t force_timeout;
 };
 
+template <int KC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CUtensorMap map_a,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_k) {
+  constexpr int kABytes = KC * kATile;
+  constexpr int kBBytes = KC * kBTile;
+  constexpr int kStageBytes = kABytes + kBBytes;
+  constexpr int kStages = kStageMem / kStageBytes;
+  static_assert(kStages <= kMaxStages, "barrier space");
   extern __shared__ uint8_t smem_raw[];
   const ProjParams& p = tp.p;
   const int warp = threadIdx.x >> 5;
@@ -76,14 +90,14 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
-  const uint32_t bar0 = base + kStages * kStageBytes;
+  const uint32_t bar0 = base + kStageMem;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * kStages + a); };
-  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 + a); };
-  const uint32_t never_bar = bar0 + 8u * (2 * kStages + 4);
-  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 5);
-  uint8_t* misc = sbase + kStages * kStageBytes + 8 * kNumBars;
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kMaxStages + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * kMaxStages + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * kMaxStages + 2 + a); };
+  const uint32_t never_bar = bar0 + 8u * (2 * kMaxStages + 4);
+  const uint32_t drain_bar = bar0 + 8u * (2 * kMaxStages + 5);
+  uint8_t* misc = sbase + kStageMem + 8 * kNumBars;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   float* wprod = reinterpret_cast<float*>(misc + 16);  // [kEpiWarps][kEpiCols] nk*nq
@@ -95,7 +109,7 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 2 * kEpiWarps * 32);  // both CTAs' epilogue threads
+      mbar_init(tempty_bar(a), 2 * kEpiWarps);       // one arrival per epilogue warp, both CTAs
     }
     mbar_init(never_bar, 1);
     mbar_init(drain_bar, 1);
@@ -142,7 +156,7 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
       const int nb = static_cast<int>(tile % tp.num_n_tiles);
       const bool is_v = nb < tp.nv_tiles;
       const int32_t yb = (is_v ? nb : nb - tp.nv_tiles) * kBN + static_cast<int32_t>(rank) * kBNh;
-      for (int kb = 0; kb < p.nh; ++kb) {
+      for (int kb = 0; kb < p.nh; kb += KC) {
         ok = wait_pair(empty_bar(stage), phase ^ 1u);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         if (lane == 0) {
@@ -153,8 +167,13 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
             pending |= 1u << stage;
             pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
           }
-          tma_load_2d_pair(sa, &map_a, kb * kBK, static_cast<int32_t>(m0), lbar, pol_a);
-          tma_load_2d_pair(sa + kABytes, is_v ? &map_v : &map_k, kb * kBK, yb, lbar, pol_w);
+          if (KC == 1) {
+            tma_load_2d_pair(sa, &map_a, kb * kBK, static_cast<int32_t>(m0), lbar, pol_a);
+            tma_load_2d_pair(sa + kABytes, is_v ? &map_v : &map_k, kb * kBK, yb, lbar, pol_w);
+          } else {
+            tma_load_3d_pair(sa, &map_a, 0, static_cast<int32_t>(m0), kb, lbar, pol_a);
+            tma_load_3d_pair(sa + kABytes, is_v ? &map_v : &map_k, 0, yb, kb, lbar, pol_w);
+          }
         }
         __syncwarp();
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -182,16 +201,19 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
         if (!ok) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
-        for (int kb = 0; kb < p.nh; ++kb) {
+        for (int kb = 0; kb < p.nh; kb += KC) {
           ok = wait_pair(full_bar(stage), phase);
           if (!ok) break;
           tc_fence_after();
           const uint32_t sa = base + stage * kStageBytes;
           const uint32_t sb = sa + kABytes;
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k)
-            tc_mma_pair(d_tmem, umma_desc_sw128(sa + k * 32), umma_desc_sw128(sb + k * 32), kIdesc,
-                        (kb > 0 || k > 0) ? 1u : 0u);
+          for (int j = 0; j < KC; ++j)
+#pragma unroll
+            for (int k = 0; k < kBK / 16; ++k)
+              tc_mma_pair(d_tmem, umma_desc_sw128(sa + j * kATile + k * 32),
+                          umma_desc_sw128(sb + j * kBTile + k * 32), kIdesc,
+                          (kb > 0 || j > 0 || k > 0) ? 1u : 0u);
           tc_commit_pair(empty_bar(stage), 0x3);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -284,8 +306,11 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
         if (live)
           p.partials[(m * p.hc + h) * p.n_tiles + cc / kEpiCols] = make_float4(dot, ssk, ssq, 0.f);
       }
+      // the warp's TMEM reads are complete (tcgen05.wait::ld) before lane 0
+      // releases the accumulator on the leader's barrier
       tc_fence_before();
-      mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
   }
@@ -306,7 +331,7 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
   }
 }
 
-constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + 8 * kNumBars + 16 + kEpiWarps * kEpiCols * 4;
+constexpr size_t kSmemBytes = 1024 + kStageMem + 8 * kNumBars + 16 + kEpiWarps * kEpiCols * 4;
 
 bool make_map2(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
                uint32_t box_rows) {
@@ -332,6 +357,33 @@ bool make_map2(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 view {64 columns, rows, cols/64 chunks} of a row-major [rows, cols]
+// matrix (chunk stride 128 bytes), box {64, box_rows, chunks}: a box lands as
+// `chunks` consecutive [box_rows x 128-byte] swizzled tiles.
+bool make_map3(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows,
+               uint32_t chunks) {
+  using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return false;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {cols * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, chunks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return reinterpret_cast<EncodeTiled>(ptr)(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KC>
+cudaError_t launch_kc(const Tc2Params& tp, const ProjParams& p, cudaStream_t s);
+
 }  // namespace
 
 // Dense A (rows == null), bf16, Dh == 64, H % 256 == 0; grid of CTA pairs.
@@ -348,22 +400,38 @@ cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s) {
   tp.num_tiles = m2 * tp.num_n_tiles;
   tp.force_timeout = (p.debug & ENGRAM_DEBUG_FORCE_TIMEOUT) ? 1 : 0;
   tp.timeout_ns = tp.force_timeout ? 20000000ull : 2000000000ull;
+  // two K-blocks per TMA box when the head count allows it
+  if (p.nh % 2 == 0) return launch_kc<2>(tp, p, s);
+  return launch_kc<1>(tp, p, s);
+}
+
+namespace {
+
+template <int KC>
+cudaError_t launch_kc(const Tc2Params& tp, const ProjParams& p, cudaStream_t s) {
   CUtensorMap map_a, map_v, map_k;
-  if (!make_map2(&map_a, p.a_src, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.M), kBK, kBM) ||
-      !make_map2(&map_v, p.w_value, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.H), kBK, kBNh) ||
-      !make_map2(&map_k, p.w_key, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.hc) * p.H, kBK, kBNh))
-    return cudaErrorInvalidValue;
+  bool ok;
+  if (KC == 1) {
+    ok = make_map2(&map_a, p.a_src, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.M), kBK, kBM) &&
+         make_map2(&map_v, p.w_value, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.H), kBK, kBNh) &&
+         make_map2(&map_k, p.w_key, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.hc) * p.H, kBK, kBNh);
+  } else {
+    ok = make_map3(&map_a, p.a_src, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.M), kBM, KC) &&
+         make_map3(&map_v, p.w_value, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.H), kBNh, KC) &&
+         make_map3(&map_k, p.w_key, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.hc) * p.H, kBNh, KC);
+  }
+  if (!ok) return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
+  static int max_pairs[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(proj_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(proj_tc2_kernel<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   // as many pairs as can be resident at once (not every SM pair need form a cluster)
-  static int max_pairs[64] = {0};
   if (dev >= 0 && dev < 64 && max_pairs[dev] == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
@@ -377,7 +445,7 @@ cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s) {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, proj_tc2_kernel, &cfg) != cudaSuccess || n <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&n, proj_tc2_kernel<KC>, &cfg) != cudaSuccess || n <= 0) {
       cudaGetLastError();  // clear; fall back to one pair per two SMs
       n = num_sms() / 2;
     }
@@ -385,9 +453,11 @@ cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s) {
   }
   int64_t pairs = (dev >= 0 && dev < 64) ? max_pairs[dev] : num_sms() / 2;
   if (pairs > tp.num_tiles) pairs = tp.num_tiles;
-  proj_tc2_kernel<<<static_cast<unsigned>(2 * pairs), kThreads, kSmemBytes, s>>>(tp, map_a, map_v, map_k);
+  proj_tc2_kernel<KC><<<static_cast<unsigned>(2 * pairs), kThreads, kSmemBytes, s>>>(tp, map_a, map_v, map_k);
   count_launch();
   return cudaGetLastError();
 }
+
+}  // namespace
 
 }  // namespace engram
