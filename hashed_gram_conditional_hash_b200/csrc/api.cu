@@ -200,6 +200,8 @@ engram_status set_error(engram_status st, const char* fmt, ...) {
   return st;
 }
 
+uint32_t debug_flags() { return g_debug.load(std::memory_order_relaxed); }
+
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 int num_sms() {

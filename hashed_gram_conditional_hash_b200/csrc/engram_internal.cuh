@@ -162,7 +162,36 @@ void count_launch(int n = 1);
 // Sets the calling thread's engram_last_error text and returns st.
 engram_status set_error(engram_status st, const char* fmt, ...);
 
+// Process-wide ENGRAM_DEBUG_* flags.
+uint32_t debug_flags();
+
+// Launch with programmatic dependent launch (PDL): the kernel may be
+// scheduled while the previous kernel on the stream is finishing; every
+// kernel of the library calls pdl_wait() before touching global memory (a
+// no-op for an ordinary launch) and pdl_trigger() once its main work is done.
+// ENGRAM_DEBUG_NO_PDL turns the attribute off.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     const Args&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (debug_flags() & ENGRAM_DEBUG_NO_PDL) ? 0 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  count_launch();
+  return e;
+}
+
 // ---------------------------------------------------------------- device side
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bits) {
   if (status != nullptr) atomicOr(status, bits);

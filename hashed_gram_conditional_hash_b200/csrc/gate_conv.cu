@@ -20,6 +20,7 @@ namespace {
 
 // -------------------------------------------------------------- gate
 __global__ void gate_kernel(const __grid_constant__ GateParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (i >= p.M * p.hc) return;
   const float4* part = p.partials + i * p.n_tiles;
@@ -158,6 +159,7 @@ __device__ __forceinline__ void load_taps(const T* row, int K, float (&w)[8][KMA
 // keeps many bytes in flight and runs at the memory system's pace.
 template <typename T, int KMAX, int HCMAX>
 __global__ void __launch_bounds__(kConvThreads) gated_conv_kernel(const __grid_constant__ ConvParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int cgs = p.H >> 3;                                   // channel groups per row
   const int64_t gid = blockIdx.x * static_cast<int64_t>(kConvThreads) + threadIdx.x;
   const int64_t row = gid / cgs;                              // token b*T + t
@@ -230,6 +232,7 @@ __global__ void __launch_bounds__(kConvThreads) gated_conv_kernel(const __grid_c
 // a handful of threads through L1/L2; DRAM sees it about once.
 template <typename T, int RUN>
 __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_constant__ ConvParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   constexpr int K = 4;
   constexpr int NW = RUN + K - 1;                 // rows in the window of a run
   // thread order: (b, residue class, run, branch, channel group), channel
@@ -321,6 +324,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
 // -------------------------------------------------------------- standalone conv
 template <typename T>
 __global__ void short_conv_kernel(const __grid_constant__ ShortConvParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const T* u = static_cast<const T*>(p.u);
   const T* w = static_cast<const T*>(p.conv_w);
   const T* st = static_cast<const T*>(p.state);
@@ -350,6 +354,7 @@ __global__ void short_conv_kernel(const __grid_constant__ ShortConvParams p) {
 // j reads index j + T > j before it is overwritten.
 template <typename T>
 __global__ void short_conv_state_kernel(const __grid_constant__ ShortConvParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (q >= static_cast<int64_t>(p.B) * p.C) return;
   const int c = static_cast<int>(q % p.C);
@@ -368,6 +373,7 @@ __global__ void short_conv_state_kernel(const __grid_constant__ ShortConvParams 
 // -------------------------------------------------------------- streaming state
 template <typename T>
 __global__ void state_advance_kernel(const __grid_constant__ StateAdvanceParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int b = blockIdx.x;
   const int64_t P = p.pos[b];
   const int n = min(p.T, p.ring_len);
@@ -388,6 +394,7 @@ __global__ void state_advance_kernel(const __grid_constant__ StateAdvanceParams 
 __global__ void state_init_kernel(int64_t* id_ring, int n_hist, uint16_t* v_ring16, float* v_ring32,
                                   float* g_ring, int64_t* pos, int64_t ring_len, int32_t B,
                                   int32_t H, int32_t hc, int64_t pad_id) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   for (int64_t i = i0; i < static_cast<int64_t>(B) * n_hist; i += stride) id_ring[i] = pad_id;
@@ -407,8 +414,7 @@ int grid_cap() { return num_sms() * 8; }
 cudaError_t launch_gate(const GateParams& p, cudaStream_t s) {
   const int64_t n = p.M * p.hc;
   if (n <= 0) return cudaSuccess;
-  gate_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
-  count_launch();
+  launch_k(gate_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, p);
   return cudaGetLastError();
 }
 
@@ -430,18 +436,17 @@ cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
     const int64_t rb = (nthreads + kConvThreads - 1) / kConvThreads;
     if (rb * kConvThreads > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit thread ids
     const unsigned g = static_cast<unsigned>(rb);
-    if (p.dtype == ENGRAM_F32) conv_run_kernel<float, kRun><<<g, kConvThreads, 0, s>>>(p);
-    else conv_run_kernel<uint16_t, kRun><<<g, kConvThreads, 0, s>>>(p);
+    if (p.dtype == ENGRAM_F32) launch_k(conv_run_kernel<float, kRun>, dim3(g), dim3(kConvThreads), 0, s, p);
+    else launch_k(conv_run_kernel<uint16_t, kRun>, dim3(g), dim3(kConvThreads), 0, s, p);
   } else if (p.K <= 4 && p.hc <= 4) {  // up to 4 taps and 4 branches
-    if (p.dtype == ENGRAM_F32) gated_conv_kernel<float, 4, 4><<<nb, kConvThreads, 0, s>>>(p);
-    else gated_conv_kernel<uint16_t, 4, 4><<<nb, kConvThreads, 0, s>>>(p);
+    if (p.dtype == ENGRAM_F32) launch_k(gated_conv_kernel<float, 4, 4>, dim3(nb), dim3(kConvThreads), 0, s, p);
+    else launch_k(gated_conv_kernel<uint16_t, 4, 4>, dim3(nb), dim3(kConvThreads), 0, s, p);
   } else {
     if (p.dtype == ENGRAM_F32)
-      gated_conv_kernel<float, ENGRAM_MAX_CONV_K, ENGRAM_MAX_HC><<<nb, kConvThreads, 0, s>>>(p);
+      launch_k(gated_conv_kernel<float, ENGRAM_MAX_CONV_K, ENGRAM_MAX_HC>, dim3(nb), dim3(kConvThreads), 0, s, p);
     else
-      gated_conv_kernel<uint16_t, ENGRAM_MAX_CONV_K, ENGRAM_MAX_HC><<<nb, kConvThreads, 0, s>>>(p);
+      launch_k(gated_conv_kernel<uint16_t, ENGRAM_MAX_CONV_K, ENGRAM_MAX_HC>, dim3(nb), dim3(kConvThreads), 0, s, p);
   }
-  count_launch();
   return cudaGetLastError();
 }
 
@@ -450,18 +455,16 @@ cudaError_t launch_short_conv(const ShortConvParams& p, cudaStream_t s) {
   if (total > 0) {
     int64_t blocks = (total + 255) / 256;
     if (blocks > grid_cap()) blocks = grid_cap();
-    if (p.dtype == ENGRAM_F32) short_conv_kernel<float><<<static_cast<int>(blocks), 256, 0, s>>>(p);
-    else short_conv_kernel<uint16_t><<<static_cast<int>(blocks), 256, 0, s>>>(p);
-    count_launch();
+    if (p.dtype == ENGRAM_F32) launch_k(short_conv_kernel<float>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, p);
+    else launch_k(short_conv_kernel<uint16_t>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (p.state != nullptr && p.T > 0 && p.K > 1) {
     const int64_t n = static_cast<int64_t>(p.B) * p.C;
     const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
-    if (p.dtype == ENGRAM_F32) short_conv_state_kernel<float><<<blocks, 256, 0, s>>>(p);
-    else short_conv_state_kernel<uint16_t><<<blocks, 256, 0, s>>>(p);
-    count_launch();
+    if (p.dtype == ENGRAM_F32) launch_k(short_conv_state_kernel<float>, dim3(blocks), dim3(256), 0, s, p);
+    else launch_k(short_conv_state_kernel<uint16_t>, dim3(blocks), dim3(256), 0, s, p);
     return cudaGetLastError();
   }
   return cudaSuccess;
@@ -469,9 +472,8 @@ cudaError_t launch_short_conv(const ShortConvParams& p, cudaStream_t s) {
 
 cudaError_t launch_state_advance(const StateAdvanceParams& p, cudaStream_t s) {
   if (p.B <= 0 || p.T <= 0) return cudaSuccess;
-  if (p.dtype == ENGRAM_F32) state_advance_kernel<float><<<p.B, 256, 0, s>>>(p);
-  else state_advance_kernel<uint16_t><<<p.B, 256, 0, s>>>(p);
-  count_launch();
+  if (p.dtype == ENGRAM_F32) launch_k(state_advance_kernel<float>, dim3(p.B), dim3(256), 0, s, p);
+  else launch_k(state_advance_kernel<uint16_t>, dim3(p.B), dim3(256), 0, s, p);
   return cudaGetLastError();
 }
 
@@ -483,11 +485,10 @@ cudaError_t launch_state_init(int64_t* id_ring, int n_hist, void* v_ring, float*
   int64_t blocks = (n + 255) / 256;
   if (blocks > grid_cap()) blocks = grid_cap();
   if (blocks < 1) blocks = 1;
-  state_init_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+  launch_k(state_init_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
       id_ring, n_hist, dt == ENGRAM_BF16 ? static_cast<uint16_t*>(v_ring) : nullptr,
       dt == ENGRAM_F32 ? static_cast<float*>(v_ring) : nullptr, g_ring, pos, ring_len, B, H, hc,
       pad_id);
-  count_launch();
   return cudaGetLastError();
 }
 

@@ -21,6 +21,7 @@ __device__ __forceinline__ int4 ld_nc_v4(const void* p) {
 }
 
 __global__ void __launch_bounds__(256) gather_v16_kernel(const __grid_constant__ GatherParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int chunks = p.row_bytes >> 4;
   const int64_t total = p.M * p.nh * chunks;
   const char* tab = static_cast<const char*>(p.table);
@@ -43,6 +44,7 @@ __global__ void __launch_bounds__(256) gather_v16_kernel(const __grid_constant__
 
 // Rows whose byte width is not a multiple of 16: 4-byte words.
 __global__ void __launch_bounds__(256) gather_v4_kernel(const __grid_constant__ GatherParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int words = p.row_bytes >> 2;
   const int64_t total = p.M * p.nh * words;
   const uint32_t* tab = static_cast<const uint32_t*>(p.table);
@@ -70,9 +72,8 @@ cudaError_t launch_gather(const GatherParams& p, cudaStream_t s) {
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;  // 8 x 256 threads per SM
   if (blocks > cap) blocks = cap;
-  if (v16) gather_v16_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(p);
-  else gather_v4_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(p);
-  count_launch();
+  if (v16) launch_k(gather_v16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, p);
+  else launch_k(gather_v4_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, p);
   return cudaGetLastError();
 }
 

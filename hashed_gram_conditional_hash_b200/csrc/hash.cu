@@ -38,6 +38,7 @@ __device__ __forceinline__ int64_t load_id(const HashParams& p, int64_t raw) {
 }
 
 __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int b = blockIdx.y;
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashP
 // the ring becomes the last n_hist ids of (old ring ++ chunk).  One thread per
 // sequence; it runs after hash_kernel on the same stream.
 __global__ void id_ring_kernel(const __grid_constant__ HashParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= p.B) return;
   int64_t* ring = p.id_ring_out + static_cast<int64_t>(b) * p.n_hist;
@@ -134,6 +136,7 @@ __device__ __forceinline__ uint64_t token_at(const HashParams& p, int b, int t) 
 // Barrett reduction by its head's prime), then the warp copies the 32 table
 // rows with every 16-byte load issued before the stores.
 __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant__ HashGatherParams g) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const HashParams& p = g.h;
   const int lane = threadIdx.x & 31;
   // rows of e (B*T*nh) stay below 2^31 (checked by the launcher): 32-bit math
@@ -182,6 +185,7 @@ __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant_
 __global__ void compress_kernel(const int64_t* __restrict__ raw, int64_t n,
                                 const int64_t* __restrict__ lookup, int64_t raw_vocab,
                                 int64_t* __restrict__ out, uint32_t* status) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     int64_t r = __ldg(raw + i);
@@ -199,14 +203,12 @@ __global__ void compress_kernel(const int64_t* __restrict__ raw, int64_t n,
 cudaError_t launch_hash(const HashParams& p, cudaStream_t s) {
   if (p.B > 0 && p.T > 0) {
     dim3 grid((p.T + 255) / 256, p.B);
-    hash_kernel<<<grid, 256, 0, s>>>(p);
-    count_launch();
+    launch_k(hash_kernel, dim3(grid), dim3(256), 0, s, p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (p.id_ring_out != nullptr && p.n_hist > 0 && p.B > 0) {
-    id_ring_kernel<<<(p.B + 127) / 128, 128, 0, s>>>(p);
-    count_launch();
+    launch_k(id_ring_kernel, dim3((p.B + 127) / 128), dim3(128), 0, s, p);
     return cudaGetLastError();
   }
   return cudaSuccess;
@@ -218,14 +220,12 @@ cudaError_t launch_hash_gather(const HashGatherParams& g, cudaStream_t s) {
   if (total > 0) {
     const int64_t blocks = (total + 255) / 256;
     if (blocks * 256 > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit row ids in the kernel
-    hash_gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(g);
-    count_launch();
+    launch_k(hash_gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   if (p.id_ring_out != nullptr && p.n_hist > 0 && p.B > 0) {
-    id_ring_kernel<<<(p.B + 127) / 128, 128, 0, s>>>(p);
-    count_launch();
+    launch_k(id_ring_kernel, dim3((p.B + 127) / 128), dim3(128), 0, s, p);
     return cudaGetLastError();
   }
   return cudaSuccess;
@@ -237,8 +237,7 @@ cudaError_t launch_compress(const int64_t* raw, int64_t n, const int64_t* lookup
   int64_t blocks = (n + 255) / 256;
   int cap = num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  compress_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(raw, n, lookup, raw_vocab, out, status);
-  count_launch();
+  launch_k(compress_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, raw, n, lookup, raw_vocab, out, status);
   return cudaGetLastError();
 }
 

@@ -20,6 +20,7 @@ constexpr int BM = 64, BN = 64, BK = 32;
 
 template <typename T>
 __global__ void __launch_bounds__(256) proj_simt_kernel(const __grid_constant__ ProjParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs[BK][BN + 4];
   const int tid = threadIdx.x;
@@ -125,9 +126,8 @@ __global__ void __launch_bounds__(256) proj_simt_kernel(const __grid_constant__ 
 cudaError_t launch_proj_simt(const ProjParams& p, cudaStream_t s) {
   if (p.M <= 0) return cudaSuccess;
   dim3 grid((1 + p.hc) * p.H / BN, static_cast<unsigned>((p.M + BM - 1) / BM));
-  if (p.dtype == ENGRAM_F32) proj_simt_kernel<float><<<grid, 256, 0, s>>>(p);
-  else proj_simt_kernel<uint16_t><<<grid, 256, 0, s>>>(p);
-  count_launch();
+  if (p.dtype == ENGRAM_F32) launch_k(proj_simt_kernel<float>, dim3(grid), dim3(256), 0, s, p);
+  else launch_k(proj_simt_kernel<uint16_t>, dim3(grid), dim3(256), 0, s, p);
   return cudaGetLastError();
 }
 

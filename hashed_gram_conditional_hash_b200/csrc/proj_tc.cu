@@ -129,6 +129,8 @@ proj_tc_kernel(const __grid_constant__ TcParams tp, const __grid_constant__ CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the set-up above overlaps the previous kernel's tail; inputs are read only now
+  pdl_wait();
   const uint64_t limit = tp.timeout_ns;
 
   if (warp == 0) {
@@ -353,6 +355,7 @@ proj_tc_kernel(const __grid_constant__ TcParams tp, const __grid_constant__ CUte
     }
   }
 
+  pdl_trigger();  // this CTA's tiles are done: the next kernel may be scheduled
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -441,8 +444,7 @@ cudaError_t launch_proj_tc(const ProjParams& p, cudaStream_t s) {
   }
   int64_t grid = num_sms();
   if (grid > tp.num_tiles) grid = tp.num_tiles;
-  proj_tc_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(tp, map_a, map_v, map_k);
-  count_launch();
+  launch_k(proj_tc_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmemBytes, s, tp, map_a, map_v, map_k);
   return cudaGetLastError();
 }
 

@@ -127,6 +127,8 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
+  // the set-up above overlaps the previous kernel's tail; inputs are read only now
+  pdl_wait();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t limit = tp.timeout_ns;
   // abort: raise the flag here and in the peer CTA, so both unwind together
@@ -315,6 +317,7 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
     }
   }
 
+  pdl_trigger();  // this CTA's tiles are done: the next kernel may be scheduled
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // neither CTA leaves while the pair may still touch its memory
@@ -453,8 +456,7 @@ cudaError_t launch_kc(const Tc2Params& tp, const ProjParams& p, cudaStream_t s) 
   }
   int64_t pairs = (dev >= 0 && dev < 64) ? max_pairs[dev] : num_sms() / 2;
   if (pairs > tp.num_tiles) pairs = tp.num_tiles;
-  proj_tc2_kernel<KC><<<static_cast<unsigned>(2 * pairs), kThreads, kSmemBytes, s>>>(tp, map_a, map_v, map_k);
-  count_launch();
+  launch_k(proj_tc2_kernel<KC>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), kSmemBytes, s, tp, map_a, map_v, map_k);
   return cudaGetLastError();
 }
 

@@ -150,6 +150,10 @@ uint64_t engram_launch_count(void);
 /* ENGRAM_DEBUG_TC_SINGLE_CTA runs the dense tensor-core projection on single
  * CTAs (128 x 256 tiles) instead of CTA pairs (256 x 256 tiles, 2-SM MMA). */
 #define ENGRAM_DEBUG_TC_SINGLE_CTA 0x8u
+/* ENGRAM_DEBUG_NO_PDL launches every kernel as an ordinary launch instead of
+ * with programmatic dependent launch (which lets a kernel be scheduled while
+ * its predecessor on the stream finishes). */
+#define ENGRAM_DEBUG_NO_PDL 0x10u
 void engram_set_debug(uint32_t flags);
 
 /* Which projection engine engram_forward / engram_gate_fuse use for cfg under
