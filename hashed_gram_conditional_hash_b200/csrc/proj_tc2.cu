@@ -22,9 +22,19 @@
 //              the barriers of both CTAs
 //   warps 2-9  epilogue on the CTA's own 128 TMEM lanes (one token row and
 //              128 columns per thread): V -> bf16, or the score partials
-//              against the hidden-state slice (loaded before the wait); the
-//              accumulator is released on the leader's barrier
+//              against the hidden-state slice; the accumulator is released
+//              on the leader's barrier
 // Accumulators are double-buffered (2 x 256 fp32 columns).
+//
+// The epilogue moves its global data through a 4 KB shared-memory tile per
+// warp (32 rows x 64 columns, 128-byte swizzle) with TMA: the hidden-state
+// slice comes in as a tensor load, V goes out as a tensor store.  Shared
+// memory and L1 share one data path with the operand stream (TMA writes and
+// the MMA's operand reads); a warp that reads or writes one 16-byte piece of
+// 32 different rows per instruction spends 32 cycles of that path on 512
+// bytes, a TMA tile plus conflict-free swizzled shared accesses about 8.  On
+// B200 the direct per-row form cost the model-shaped projection ~15 us of
+// its ~74 us.
 //
 // TMA delivers a fixed number of boxes per SM per second (measured on B200:
 // 16 KB boxes stream at ~56 GB/s per SM, 32 KB boxes at ~112 GB/s, at any
@@ -59,7 +69,11 @@ constexpr int kEpiCols = kBN / 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_bf16(2 * kBM, kBN);
 constexpr int kMaxStages = 6;
-constexpr int kNumBars = 2 * kMaxStages + 2 + 2 + 2;  // full, empty, tfull, tempty, never, drain
+constexpr int kEpiRows = 32;                // token rows per epilogue warp
+constexpr int kXCols = 64;                  // columns per staged tile (128 bytes of bf16)
+constexpr int kXBytes = kEpiRows * kXCols * 2;   // 4 KB staging tile per epilogue warp
+// full, empty, tfull, tempty, never, drain, one hidden-state barrier per epilogue warp
+constexpr int kNumBars = 2 * kMaxStages + 2 + 2 + 2 + kEpiWarps;
 
 struct Tc2Params {
   ProjParams p;
@@ -72,7 +86,8 @@ struct Tc2Params {
 template <int KC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CUtensorMap map_a,
-                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_k) {
+                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_k,
+                const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_vo) {
   constexpr int kABytes = KC * kATile;
   constexpr int kBBytes = KC * kBTile;
   constexpr int kStageBytes = kABytes + kBBytes;
@@ -90,17 +105,18 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
-  const uint32_t bar0 = base + kStageMem;
+  const uint32_t xbuf0 = base + kStageMem;                 // epilogue staging tiles
+  const uint32_t bar0 = xbuf0 + kEpiWarps * kXBytes;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kMaxStages + s); };
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * kMaxStages + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * kMaxStages + 2 + a); };
   const uint32_t never_bar = bar0 + 8u * (2 * kMaxStages + 4);
   const uint32_t drain_bar = bar0 + 8u * (2 * kMaxStages + 5);
-  uint8_t* misc = sbase + kStageMem + 8 * kNumBars;
+  auto xbar = [&](int w) { return bar0 + 8u * (2 * kMaxStages + 6 + w); };
+  uint8_t* misc = sbase + kStageMem + kEpiWarps * kXBytes + 8 * kNumBars;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
-  float* wprod = reinterpret_cast<float*>(misc + 16);  // [kEpiWarps][kEpiCols] nk*nq
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -113,6 +129,7 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
     }
     mbar_init(never_bar, 1);
     mbar_init(drain_bar, 1);
+    for (int w = 0; w < kEpiWarps; ++w) mbar_init(xbar(w), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -145,6 +162,8 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_v)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_k)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_q)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_vo)) : "memory");
     }
     uint64_t pol_w, pol_a;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_w));
@@ -231,83 +250,115 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
     const int quad = warp & 3;               // TMEM lanes 32*quad .. +31
-    const int half = (warp - 2) >> 2;        // column half of the tile
-    const int row = quad * 32 + lane;
+    const int half = ew >> 2;                // column half of the tile
+    const uint32_t xb = xbuf0 + ew * kXBytes;
+    const uint32_t qbar = xbar(ew);
+    uint32_t q_par = 0;                      // parity of the next hidden-state fill
+    bool q_inflight = false;                 // a fill was issued and not yet waited for
     int acc = 0;
     uint32_t acc_phase = 0;
-    const uint16_t* hid = static_cast<const uint16_t*>(p.hidden);
     const uint16_t* nk = static_cast<const uint16_t*>(p.norm_key);
     const uint16_t* nq = static_cast<const uint16_t*>(p.norm_query);
-    uint16_t* V = static_cast<uint16_t*>(p.V);
-    float* wp = wprod + (warp - 2) * kEpiCols;
+    // this warp's hidden-state slice, 64 columns at a time: {column, branch, token}
+    auto fill_q = [&](int col, int h, int32_t tok) {
+      if (lane == 0) {
+        bulk_wait_group_read0();             // a V store from this tile has left it
+        mbar_arrive_expect_tx(qbar, kXBytes);
+        tma_load_3d(xb, &map_q, col, h, tok, qbar);
+      }
+      q_inflight = true;
+    };
     for (int64_t tile = pair; tile < tp.num_tiles; tile += npairs) {
-      const int64_t m = (tile / tp.num_n_tiles) * (2 * kBM) + rank * kBM + row;
+      const int64_t tok0 = (tile / tp.num_n_tiles) * (2 * kBM) + rank * kBM + quad * kEpiRows;
+      const int64_t m = tok0 + lane;
       const int nb = static_cast<int>(tile % tp.num_n_tiles);
       const bool live = m < p.M;
       const bool is_v = nb < tp.nv_tiles;
       const int kt = nb - tp.nv_tiles;
       const int h = is_v ? 0 : kt / tp.nv_tiles;
       const int c0 = is_v ? nb * kBN : (kt - h * tp.nv_tiles) * kBN;  // first column in H
-      const int cc = c0 + half * kEpiCols;                               // this thread's first
-      uint4 qv[kEpiCols / 8];
+      const int cc = c0 + half * kEpiCols;                               // this warp's first
       if (!is_v) {
-        const uint4* qsrc = reinterpret_cast<const uint4*>(hid + (m * p.hc + h) * p.H + cc);
-#pragma unroll
-        for (int q = 0; q < kEpiCols / 8; ++q) qv[q] = live ? __ldg(qsrc + q) : make_uint4(0, 0, 0, 0);
-        const int64_t wi = static_cast<int64_t>(h) * p.H + cc + 4 * lane;
-        const uint2 a = __ldg(reinterpret_cast<const uint2*>(nk + wi));
-        const uint2 b = __ldg(reinterpret_cast<const uint2*>(nq + wi));
-        __syncwarp();  // every lane is done reading the previous tile's values
-        float4 w4;
-        w4.x = __uint_as_float(a.x << 16) * __uint_as_float(b.x << 16);
-        w4.y = __uint_as_float(a.x & 0xffff0000u) * __uint_as_float(b.x & 0xffff0000u);
-        w4.z = __uint_as_float(a.y << 16) * __uint_as_float(b.y << 16);
-        w4.w = __uint_as_float(a.y & 0xffff0000u) * __uint_as_float(b.y & 0xffff0000u);
-        reinterpret_cast<float4*>(wp)[lane] = w4;
-        __syncwarp();
+        fill_q(cc, h, static_cast<int32_t>(tok0));
+        if (lane == 0) tma_prefetch_l2_3d(&map_q, cc + kXCols, h, static_cast<int32_t>(tok0));
       }
       const bool ok = wait_pair(tfull_bar(acc), acc_phase);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * kBN + half * kEpiCols);
-      if (is_v) {
-        uint16_t* vrow = V + m * p.H + cc;
+      bool fine = true;
+      if (is_v && tok0 < p.M) {  // (a warp whose rows all lie past M stores nothing)
+        // V -> bf16 into the staging tile (swizzled rows), then one tensor store per 64 columns
 #pragma unroll 1
-        for (int ch = 0; ch < kEpiCols / 32; ++ch) {
-          float v[32];
-          tmem_ld32(taddr + ch * 32, v);
-          if (live) {
-            uint4* dst = reinterpret_cast<uint4*>(vrow + ch * 32);
+        for (int f = 0; f < kEpiCols / kXCols; ++f) {
+          if (lane == 0) bulk_wait_group_read0();  // the previous store has left the tile
+          __syncwarp();
+#pragma unroll
+          for (int c2 = 0; c2 < kXCols / 32; ++c2) {
+            float v[32];
+            tmem_ld32(taddr + (f * kXCols + c2 * 32), v);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              dst[q] = make_uint4(bf16x2(v[8 * q + 0], v[8 * q + 1]), bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                  bf16x2(v[8 * q + 4], v[8 * q + 5]), bf16x2(v[8 * q + 6], v[8 * q + 7]));
+              st_shared_v4(xb + sw128_offset(lane, c2 * 4 + q),
+                           make_uint4(bf16x2(v[8 * q + 0], v[8 * q + 1]), bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                      bf16x2(v[8 * q + 4], v[8 * q + 5]), bf16x2(v[8 * q + 6], v[8 * q + 7])));
+          }
+          fence_proxy_async();  // the tile's generic writes are visible to the tensor store
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_vo, xb, cc + f * kXCols, static_cast<int32_t>(tok0));
+            bulk_commit_group();
           }
         }
-      } else {
+      } else if (!is_v) {
         float dot = 0.f, ssk = 0.f, ssq = 0.f;
+#pragma unroll 1
+        for (int f = 0; f < kEpiCols / kXCols && fine; ++f) {
+          if (f > 0) {
+            __syncwarp();  // every lane has consumed the previous fill
+            fill_q(cc + f * kXCols, h, static_cast<int32_t>(tok0));
+          }
+          fine = __all_sync(0xffffffffu, wait_pair(qbar, q_par));
+          if (!fine) break;
+          q_inflight = false;
+          q_par ^= 1u;
 #pragma unroll
-        for (int ch = 0; ch < kEpiCols / 32; ++ch) {
-          float k[32];
-          tmem_ld32(taddr + ch * 32, k);
-          const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qv[4 * ch]);
+          for (int c2 = 0; c2 < kXCols / 32; ++c2) {
+            const int col = cc + f * kXCols + c2 * 32;
+            float k[32];
+            tmem_ld32(taddr + (f * kXCols + c2 * 32), k);
+            const uint4* nk4 = reinterpret_cast<const uint4*>(nk + static_cast<int64_t>(h) * p.H + col);
+            const uint4* nq4 = reinterpret_cast<const uint4*>(nq + static_cast<int64_t>(h) * p.H + col);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float q0 = __uint_as_float(qw[i] << 16), q1 = __uint_as_float(qw[i] & 0xffff0000u);
-            const float k0 = k[2 * i], k1 = k[2 * i + 1];
-            dot = fmaf(k0 * wp[ch * 32 + 2 * i], q0, dot);
-            dot = fmaf(k1 * wp[ch * 32 + 2 * i + 1], q1, dot);
-            ssk = fmaf(k0, k0, ssk);
-            ssk = fmaf(k1, k1, ssk);
-            ssq = fmaf(q0, q0, ssq);
-            ssq = fmaf(q1, q1, ssq);
+            for (int q = 0; q < 4; ++q) {
+              const uint4 qq = ld_shared_v4(xb + sw128_offset(lane, c2 * 4 + q));
+              const uint4 ka = __ldg(nk4 + q), qa = __ldg(nq4 + q);
+              const uint32_t qw[4] = {qq.x, qq.y, qq.z, qq.w};
+              const uint32_t kw[4] = {ka.x, ka.y, ka.z, ka.w};
+              const uint32_t nw[4] = {qa.x, qa.y, qa.z, qa.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float q0 = __uint_as_float(qw[i] << 16), q1 = __uint_as_float(qw[i] & 0xffff0000u);
+                const float w0 = __uint_as_float(kw[i] << 16) * __uint_as_float(nw[i] << 16);
+                const float w1 = __uint_as_float(kw[i] & 0xffff0000u) * __uint_as_float(nw[i] & 0xffff0000u);
+                const float k0 = k[8 * q + 2 * i], k1 = k[8 * q + 2 * i + 1];
+                dot = fmaf(k0 * w0, q0, dot);
+                dot = fmaf(k1 * w1, q1, dot);
+                ssk = fmaf(k0, k0, ssk);
+                ssk = fmaf(k1, k1, ssk);
+                ssq = fmaf(q0, q0, ssq);
+                ssq = fmaf(q1, q1, ssq);
+              }
+            }
           }
         }
-        if (live)
+        if (fine && live)
           p.partials[(m * p.hc + h) * p.n_tiles + cc / kEpiCols] = make_float4(dot, ssk, ssq, 0.f);
       }
+      if (!fine) break;
       // the warp's TMEM reads are complete (tcgen05.wait::ld) before lane 0
       // releases the accumulator on the leader's barrier
       tc_fence_before();
@@ -315,6 +366,15 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
       if (lane == 0) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    // outstanding transfers of this warp end before its shared memory is released
+    if (lane == 0) {
+      bulk_wait_group0();
+      if (q_inflight) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(qbar, q_par) && globaltimer() - t0 < limit) {}
+      }
+    }
+    __syncwarp();
   }
 
   pdl_trigger();  // this CTA's tiles are done: the next kernel may be scheduled
@@ -334,7 +394,8 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
   }
 }
 
-constexpr size_t kSmemBytes = 1024 + kStageMem + 8 * kNumBars + 16 + kEpiWarps * kEpiCols * 4;
+constexpr size_t kSmemBytes = 1024 + kStageMem + kEpiWarps * kXBytes + 8 * kNumBars + 16;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 bool make_map2(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
                uint32_t box_rows) {
@@ -384,6 +445,29 @@ bool make_map3(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 view {H columns, hc branches, M tokens} of the hidden states
+// [M, hc, H], box {64, 1, 32}: one epilogue warp's 32 tokens x 64 columns of
+// one branch, landing as a 128-byte-swizzled 32 x 128-byte tile.
+bool make_map_hidden(CUtensorMap* map, const void* base, uint64_t H, uint64_t hc, uint64_t M) {
+  using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return false;
+  cuuint64_t dims[3] = {H, hc, M};
+  cuuint64_t strides[2] = {H * 2, hc * H * 2};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kXCols), 1, static_cast<cuuint32_t>(kEpiRows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return reinterpret_cast<EncodeTiled>(ptr)(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int KC>
 cudaError_t launch_kc(const Tc2Params& tp, const ProjParams& p, cudaStream_t s);
 
@@ -423,6 +507,10 @@ cudaError_t launch_kc(const Tc2Params& tp, const ProjParams& p, cudaStream_t s) 
          make_map3(&map_v, p.w_value, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.H), kBNh, KC) &&
          make_map3(&map_k, p.w_key, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.hc) * p.H, kBNh, KC);
   }
+  CUtensorMap map_q, map_vo;
+  ok = ok && make_map_hidden(&map_q, p.hidden, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.hc),
+                             static_cast<uint64_t>(p.M)) &&
+       make_map2(&map_vo, p.V, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.M), kXCols, kEpiRows);
   if (!ok) return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
   static int max_pairs[64] = {0};
@@ -456,7 +544,8 @@ cudaError_t launch_kc(const Tc2Params& tp, const ProjParams& p, cudaStream_t s) 
   }
   int64_t pairs = (dev >= 0 && dev < 64) ? max_pairs[dev] : num_sms() / 2;
   if (pairs > tp.num_tiles) pairs = tp.num_tiles;
-  launch_k(proj_tc2_kernel<KC>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), kSmemBytes, s, tp, map_a, map_v, map_k);
+  launch_k(proj_tc2_kernel<KC>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), kSmemBytes, s, tp, map_a, map_v, map_k,
+           map_q, map_vo);
   return cudaGetLastError();
 }
 
