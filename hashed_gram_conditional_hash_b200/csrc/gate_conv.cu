@@ -223,13 +223,41 @@ __global__ void __launch_bounds__(kConvThreads) gated_conv_kernel(const __grid_c
   }
 }
 
+// Eight channels as four channel pairs, for the packed two-lane fp32
+// instructions (__fmul2_rn / __ffma2_rn: two IEEE fp32 operations each, the
+// same roundings as the scalar ones).
+template <typename T> struct Pair8;
+template <> struct Pair8<uint16_t> {
+  static __device__ __forceinline__ void unpack(const uint4& w, float2 (&v)[4]) {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xffff0000u));
+  }
+  static __device__ __forceinline__ void store(uint16_t* p, const float2 (&v)[4]) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0].x, v[0].y), pack_bf16x2(v[1].x, v[1].y),
+                                              pack_bf16x2(v[2].x, v[2].y), pack_bf16x2(v[3].x, v[3].y));
+  }
+};
+template <> struct Pair8<float> {
+  static __device__ __forceinline__ void unpack(const F8& w, float2 (&v)[4]) {
+    v[0] = make_float2(w.a.x, w.a.y); v[1] = make_float2(w.a.z, w.a.w);
+    v[2] = make_float2(w.b.x, w.b.y); v[3] = make_float2(w.b.z, w.b.w);
+  }
+  static __device__ __forceinline__ void store(float* p, const float2 (&v)[4]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0].x, v[0].y, v[1].x, v[1].y);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[2].x, v[2].y, v[3].x, v[3].y);
+  }
+};
+
 // Run form for the pages' kernel of K = 4 taps.  The taps of position t are
 // t - 3 dil, t - 2 dil, t - dil, t: all in t's residue class mod dil.  A
 // thread owns 8 channels of one branch along a run of RUN consecutive
 // positions of one residue class: it issues every load of the run at once
 // (RUN + 3 V rows of 16 bytes, kept packed, and their gates), then produces
-// RUN outputs from registers with that branch's taps.  Each V row is read by
-// a handful of threads through L1/L2; DRAM sees it about once.
+// RUN outputs from registers with that branch's taps, two channels per
+// instruction.  A run whose window lies inside the chunk (all but the first
+// runs of a sequence) takes a path with no per-row checks.  Each V row is
+// read by a handful of threads through L1/L2; DRAM sees it about once.
 template <typename T, int RUN>
 __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_constant__ ConvParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
@@ -255,68 +283,91 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
   const int c = (rem - h * cgs) * 8;
   const int t_first = cls + p.dil * (jr * RUN);   // first output position of the run
   if (t_first >= p.T) return;
+  const int t0 = t_first - (K - 1) * p.dil;       // window row 0
   const T* V = static_cast<const T*>(p.V);
   const T* vr = static_cast<const T*>(p.v_ring);
   T* Y = static_cast<T*>(p.Y);
   const int64_t seq = static_cast<int64_t>(b) * p.T;
-  const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) : 0;
 
-  // window row k is position t_first + (k - 3) * dil
   typename Raw8<T>::type vraw[NW];
   float gw[NW];
+  if (t0 >= 0 && t_first + (RUN - 1) * p.dil < p.T) {
+    // the window lies inside the chunk
+    const T* vp = V + (seq + t0) * p.H + c;
+    const float* gp = p.g + (seq + t0) * p.hc + h;
+    const int64_t vs = static_cast<int64_t>(p.dil) * p.H;
+    const int gs = p.dil * p.hc;
 #pragma unroll
-  for (int k = 0; k < NW; ++k) {
-    const int tp = t_first + (k - (K - 1)) * p.dil;
-    const float* gsrc = nullptr;
-    const T* vsrc = nullptr;
-    if (tp >= 0 && tp < p.T) {
-      gsrc = p.g + (seq + tp) * p.hc + h;
-      vsrc = V + (seq + tp) * p.H + c;
-    } else if (tp < 0 && vr != nullptr && P + tp >= 0) {
-      const int64_t rb = static_cast<int64_t>(b) * p.ring_len + (P + tp) % p.ring_len;
-      gsrc = p.g_ring + rb * p.hc + h;
-      vsrc = vr + rb * p.H + c;
+    for (int k = 0; k < NW; ++k) {
+      vraw[k] = Raw8<T>::load(vp + k * vs);
+      gw[k] = __ldg(gp + k * gs);
     }
-    if (vsrc != nullptr) {
-      vraw[k] = Raw8<T>::load(vsrc);
-      gw[k] = __ldg(gsrc);
-    } else {
-      vraw[k] = Raw8<T>::zero();
-      gw[k] = 0.f;
+  } else {
+    const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) : 0;
+#pragma unroll
+    for (int k = 0; k < NW; ++k) {
+      const int tp = t0 + k * p.dil;
+      const float* gsrc = nullptr;
+      const T* vsrc = nullptr;
+      if (tp >= 0 && tp < p.T) {
+        gsrc = p.g + (seq + tp) * p.hc + h;
+        vsrc = V + (seq + tp) * p.H + c;
+      } else if (tp < 0 && vr != nullptr && P + tp >= 0) {
+        const int64_t rb = static_cast<int64_t>(b) * p.ring_len + (P + tp) % p.ring_len;
+        gsrc = p.g_ring + rb * p.hc + h;
+        vsrc = vr + rb * p.H + c;
+      }
+      if (vsrc != nullptr) {
+        vraw[k] = Raw8<T>::load(vsrc);
+        gw[k] = __ldg(gsrc);
+      } else {
+        vraw[k] = Raw8<T>::zero();
+        gw[k] = 0.f;
+      }
     }
   }
-  float w[8][K];
-  load_taps<T, K>(static_cast<const T*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, K, w);
+  float2 w2[4][K];                                // [channel pair][tap]
+  {
+    float w[8][K];
+    load_taps<T, K>(static_cast<const T*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, K, w);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < K; ++i) w2[j][i] = make_float2(w[2 * j][i], w[2 * j + 1][i]);
+  }
   // sliding window of U = g * V: each row is unpacked and scaled once
-  float u[K][8];
+  float2 u[K][4];
 #pragma unroll
   for (int k = 0; k < K - 1; ++k) {
-    float v[8];
-    Raw8<T>::unpack(vraw[k], v);
+    float2 v[4];
+    Pair8<T>::unpack(vraw[k], v);
+    const float2 g2 = make_float2(gw[k], gw[k]);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) u[k + 1][j] = gw[k] * v[j];
+    for (int j = 0; j < 4; ++j) u[k + 1][j] = __fmul2_rn(g2, v[j]);
   }
+  T* yp = Y + ((seq + t_first) * p.hc + h) * p.H + c;
+  const int64_t ys = static_cast<int64_t>(p.dil) * p.hc * p.H;
 #pragma unroll
   for (int q = 0; q < RUN; ++q) {
 #pragma unroll
     for (int i = 0; i < K - 1; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) u[i][j] = u[i + 1][j];
-    float v[8];
-    Raw8<T>::unpack(vraw[q + K - 1], v);
+      for (int j = 0; j < 4; ++j) u[i][j] = u[i + 1][j];
+    float2 v[4];
+    Pair8<T>::unpack(vraw[q + K - 1], v);
+    const float2 g2 = make_float2(gw[q + K - 1], gw[q + K - 1]);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) u[K - 1][j] = gw[q + K - 1] * v[j];    // U(t)
-    const int t = t_first + q * p.dil;
-    if (t < p.T) {
-      float acc[8];
+    for (int j = 0; j < 4; ++j) u[K - 1][j] = __fmul2_rn(g2, v[j]);    // U(t)
+    if (t_first + q * p.dil < p.T) {
+      float2 acc[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float a = u[K - 1][j];
+      for (int j = 0; j < 4; ++j) {
+        float2 a = u[K - 1][j];
 #pragma unroll
-        for (int i = 0; i < K; ++i) a = fmaf(w[j][i], u[i][j], a);
+        for (int i = 0; i < K; ++i) a = __ffma2_rn(w2[j][i], u[i][j], a);
         acc[j] = a;
       }
-      Vec8<T>::store(Y + ((seq + t) * p.hc + h) * p.H + c, acc);
+      Pair8<T>::store(yp + q * ys, acc);
     }
   }
 }
