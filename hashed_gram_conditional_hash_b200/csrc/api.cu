@@ -487,6 +487,7 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
     if ((hp.n_hist > 0 && state->id_ring == nullptr) || state->v_ring == nullptr ||
         state->g_ring == nullptr || state->pos == nullptr)
       return fail(ENGRAM_ERR_INVALID_ARG, "a state array is NULL");
+    if (!aligned16(state->v_ring)) return fail(ENGRAM_ERR_INVALID_ARG, "state v_ring must be 16-byte aligned");
   }
   const ForwardLayout L = forward_layout(cfg, M);
   if (ws_bytes < L.st.end)

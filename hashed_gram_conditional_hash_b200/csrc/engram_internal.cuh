@@ -108,6 +108,26 @@ struct GateParams {
 };
 cudaError_t launch_gate(const GateParams& p, cudaStream_t s);
 
+// Division of a non-negative 32-bit integer n < 2^31 by a divisor d fixed
+// at launch: q = (umulhi(n, mul) + n) >> shift, with shift = ceil(log2 d)
+// and mul = floor(2^32 (2^shift - d) / d) + 1 (the invariant-divisor method
+// of Granlund and Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994).  umulhi(n, mul) < n keeps the sum below 2^32.
+struct FastDiv {
+  uint32_t d = 1, mul = 1, shift = 0;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.shift = 0;
+  while ((static_cast<uint64_t>(1) << f.shift) < d) ++f.shift;
+  f.mul = static_cast<uint32_t>(((static_cast<uint64_t>(1) << 32) * ((static_cast<uint64_t>(1) << f.shift) - d)) / d + 1);
+  return f;
+}
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.mul) + n) >> f.shift;
+}
+
 // Gated value + short conv + residual (a8, a9) from V and the gates.
 //   Y[b,t,h,c] = U(t) + sum_i w[h*H+c, i] U(t - (K-1-i) dil),  U(t) = g[t,h] V[t,c]
 // Positions before the chunk come from the state rings (if any) or are zero.
@@ -123,6 +143,8 @@ struct ConvParams {
   int32_t ring_len;
   int32_t B, T, H, hc, K, dil;
   engram_dtype dtype;
+  // thread decode of the run form (set by launch_gated_conv)
+  FastDiv div_b, div_cls, div_run, div_cg;
 };
 cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s);
 
@@ -246,6 +268,33 @@ __device__ __forceinline__ float gate_from_score(float s, float gate_eps) {
   float sg = (s > 0.f) ? 1.f : ((s < 0.f) ? -1.f : 0.f);
   float z = sqrtf(a) * sg;
   return 1.f / (1.f + expf(-z));
+}
+
+// Gate of one (token, branch) from its n_tiles score partials
+// (sum K*nk*nq*Q, sum K^2, sum Q^2 per column tile), summed in tile order:
+//   s = dot / (sqrt(ssk/H + eps) sqrt(ssq/H + eps) sqrt(H)),  g = gate(s).
+__device__ __forceinline__ float gate_from_partials(const float4* part, int n_tiles, int H, float rms_eps,
+                                                    float gate_eps) {
+  float dot = 0.f, ssk = 0.f, ssq = 0.f;
+  int t = 0;
+  for (; t + 8 <= n_tiles; t += 8) {   // eight independent loads in flight
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldg(part + t + u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) { dot += v[u].x; ssk += v[u].y; ssq += v[u].z; }
+  }
+  for (; t < n_tiles; ++t) {
+    const float4 v = __ldg(part + t);
+    dot += v.x;
+    ssk += v.y;
+    ssq += v.z;
+  }
+  const float invH = 1.f / static_cast<float>(H);
+  const float rk = sqrtf(ssk * invH + rms_eps);
+  const float rq = sqrtf(ssq * invH + rms_eps);
+  const float s = dot / (rk * rq * sqrtf(static_cast<float>(H)));
+  return gate_from_score(s, gate_eps);
 }
 
 }  // namespace engram

@@ -23,27 +23,7 @@ __global__ void gate_kernel(const __grid_constant__ GateParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (i >= p.M * p.hc) return;
-  const float4* part = p.partials + i * p.n_tiles;
-  float dot = 0.f, ssk = 0.f, ssq = 0.f;
-  int t = 0;
-  for (; t + 8 <= p.n_tiles; t += 8) {   // eight independent loads in flight
-    float4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = __ldg(part + t + u);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) { dot += v[u].x; ssk += v[u].y; ssq += v[u].z; }
-  }
-  for (; t < p.n_tiles; ++t) {
-    const float4 v = __ldg(part + t);
-    dot += v.x;
-    ssk += v.y;
-    ssq += v.z;
-  }
-  const float invH = 1.f / static_cast<float>(p.H);
-  const float rk = sqrtf(ssk * invH + p.rms_eps);
-  const float rq = sqrtf(ssq * invH + p.rms_eps);
-  const float s = dot / (rk * rq * sqrtf(static_cast<float>(p.H)));
-  const float g = gate_from_score(s, p.gate_eps);
+  const float g = gate_from_partials(p.partials + i * p.n_tiles, p.n_tiles, p.H, p.rms_eps, p.gate_eps);
   p.g[i] = g;
   if (p.g_copy != nullptr) p.g_copy[i] = g;
 }
@@ -264,24 +244,19 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
   constexpr int K = 4;
   constexpr int NW = RUN + K - 1;                 // rows in the window of a run
   // thread order: (b, residue class, run, branch, channel group), channel
-  // group fastest; the launcher keeps the thread count below 2^31, so the
-  // decode is 32-bit
-  const int cgs = p.H >> 3;
-  const int gid = static_cast<int>(blockIdx.x) * kConvThreads + static_cast<int>(threadIdx.x);
-  const int runs_per_class = (p.T + p.dil * RUN - 1) / (p.dil * RUN);
-  const int per_run = p.hc * cgs;
-  const int per_cls = runs_per_class * per_run;
-  const int per_b = p.dil * per_cls;
-  if (gid >= per_b * p.B) return;
-  const int b = gid / per_b;
-  int rem = gid - b * per_b;
-  const int cls = rem / per_cls;
-  rem -= cls * per_cls;
-  const int jr = rem / per_run;
-  rem -= jr * per_run;
-  const int h = rem / cgs;
-  const int c = (rem - h * cgs) * 8;
-  const int t_first = cls + p.dil * (jr * RUN);   // first output position of the run
+  // group fastest; the launcher keeps the thread count below 2^31 and
+  // supplies the divisors (per sequence, per class, per run, per branch)
+  const uint32_t gid = blockIdx.x * kConvThreads + threadIdx.x;
+  if (gid >= p.div_b.d * static_cast<uint32_t>(p.B)) return;
+  const uint32_t b = fast_div(gid, p.div_b);
+  uint32_t rem = gid - b * p.div_b.d;
+  const uint32_t cls = fast_div(rem, p.div_cls);
+  rem -= cls * p.div_cls.d;
+  const uint32_t jr = fast_div(rem, p.div_run);
+  rem -= jr * p.div_run.d;
+  const int h = static_cast<int>(fast_div(rem, p.div_cg));
+  const int c = static_cast<int>(rem - h * p.div_cg.d) * 8;
+  const int t_first = static_cast<int>(cls + p.dil * (jr * RUN));   // first output position of the run
   if (t_first >= p.T) return;
   const int t0 = t_first - (K - 1) * p.dil;       // window row 0
   const T* V = static_cast<const T*>(p.V);
@@ -368,6 +343,146 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
         acc[j] = a;
       }
       Pair8<T>::store(yp + q * ys, acc);
+    }
+  }
+}
+
+// Tile form for K = 4 taps, bfloat16, 256-channel slices.  A block owns
+// kTileT consecutive positions of one sequence and one 256-channel slice, all
+// branches (one warp per branch, 8 channels per lane).  It first copies the V
+// rows of the tile and of its 3*dil-row halo into shared memory with cp.async
+// (one 16-byte piece per request, no registers held; halo rows before the
+// chunk come from the state ring or are zero) and their gates, then every
+// warp walks each residue class mod dil through shared memory with a
+// four-slot window of U = g*V in registers: per position one conflict-free
+// 16-byte shared load, 8 channels of U, 4 taps two channels per instruction
+// (__ffma2_rn), one coalesced 16-byte store of Y.  Global memory sees each V
+// row once per tile (plus the halo) and each Y element once.
+constexpr int kTileT = 32;        // positions per block
+constexpr int kTileC = 256;       // channels per block (512 bytes of a bf16 row)
+constexpr int kTileMaxDil = 32;   // longer halos take the run form
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_tile_kernel(const __grid_constant__ ConvParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  constexpr int K = 4;
+  extern __shared__ __align__(16) uint8_t conv_smem[];
+  const int tiles_per_seq = (p.T + kTileT - 1) / kTileT;
+  const int b = static_cast<int>(blockIdx.x) / tiles_per_seq;
+  const int t0 = (static_cast<int>(blockIdx.x) - b * tiles_per_seq) * kTileT;
+  const int c0 = static_cast<int>(blockIdx.y) * kTileC;
+  const int halo = (K - 1) * p.dil;
+  const int n_out = min(kTileT, p.T - t0);
+  const int nr = n_out + halo;                      // smem row r is position t0 - halo + r
+  const int nthreads = static_cast<int>(blockDim.x);
+  const int tid = static_cast<int>(threadIdx.x);
+  const uint16_t* V = static_cast<const uint16_t*>(p.V);
+  const uint16_t* vr = static_cast<const uint16_t*>(p.v_ring);
+  const int64_t seq = static_cast<int64_t>(b) * p.T;
+  const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) : 0;
+  const uint32_t sV = static_cast<uint32_t>(__cvta_generic_to_shared(conv_smem));
+  float* sG = reinterpret_cast<float*>(conv_smem + static_cast<size_t>(nr) * (kTileC * 2));
+
+  // ---- stage V rows (32 pieces of 16 bytes each) and gates
+  for (int i = tid; i < nr * 32; i += nthreads) {
+    const int r = i >> 5, k = i & 31;
+    const int t = t0 - halo + r;
+    const uint32_t dst = sV + static_cast<uint32_t>(r * (kTileC * 2) + k * 16);
+    if (t >= 0) {
+      cp_async16(dst, V + (seq + t) * p.H + c0 + k * 8);
+    } else if (vr != nullptr && P + t >= 0) {
+      const int64_t rb = static_cast<int64_t>(b) * p.ring_len + (P + t) % p.ring_len;
+      cp_async16(dst, vr + rb * p.H + c0 + k * 8);
+    } else {
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+    }
+  }
+  for (int i = tid; i < nr * p.hc; i += nthreads) {
+    const int r = i / p.hc, hh = i - r * p.hc;
+    const int t = t0 - halo + r;
+    float gv = 0.f;
+    if (t >= 0) {
+      gv = __ldg(p.g + (seq + t) * p.hc + hh);
+    } else if (vr != nullptr && P + t >= 0) {
+      gv = __ldg(p.g_ring + (static_cast<int64_t>(b) * p.ring_len + (P + t) % p.ring_len) * p.hc + hh);
+    }
+    sG[i] = gv;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+
+  // ---- one warp per branch, 8 channels per lane
+  const int h = tid >> 5, lane = tid & 31;
+  if (h >= p.hc) return;
+  const int c = c0 + lane * 8;
+  float2 w2[4][K];                                // [channel pair][tap]
+  {
+    float w[8][K];
+    load_taps<uint16_t, K>(static_cast<const uint16_t*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, K, w);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < K; ++i) w2[j][i] = make_float2(w[2 * j][i], w[2 * j + 1][i]);
+  }
+  const uint32_t lane_off = sV + static_cast<uint32_t>(lane * 16);
+  auto U = [&](int r, float2 (&u)[4]) {            // U of smem row r, this lane's channels
+    uint4 raw;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
+                 : "r"(lane_off + static_cast<uint32_t>(r * (kTileC * 2))));
+    float2 v[4];
+    Pair8<uint16_t>::unpack(raw, v);
+    const float gg = sG[r * p.hc + h];
+    const float2 g2 = make_float2(gg, gg);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) u[j] = __fmul2_rn(g2, v[j]);
+  };
+  uint16_t* Y = static_cast<uint16_t*>(p.Y);
+  const int64_t ystep = static_cast<int64_t>(p.dil) * p.hc * p.H;
+  // output at row r (position t0 - halo + r) from taps in slots A (r - 3 dil),
+  // B (r - 2 dil), C (r - dil) and D (r, written here)
+  auto out = [&](uint16_t* yp, const float2 (&A)[4], const float2 (&Bv)[4], const float2 (&C)[4],
+                 const float2 (&D)[4]) {
+    float2 acc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 a = D[j];
+      a = __ffma2_rn(w2[j][0], A[j], a);
+      a = __ffma2_rn(w2[j][1], Bv[j], a);
+      a = __ffma2_rn(w2[j][2], C[j], a);
+      a = __ffma2_rn(w2[j][3], D[j], a);
+      acc[j] = a;
+    }
+    Pair8<uint16_t>::store(yp, acc);
+  };
+  for (int cls = 0; cls < p.dil && cls < n_out; ++cls) {
+    float2 ua[4], ub[4], uc[4], ud[4];
+    U(cls, ua);
+    U(cls + p.dil, ub);
+    U(cls + 2 * p.dil, uc);
+    uint16_t* yp = Y + ((seq + t0 + cls) * p.hc + h) * p.H + c;
+    for (int r = cls + halo; r < nr; r += 4 * p.dil) {
+      U(r, ud);
+      out(yp, ua, ub, uc, ud);
+      yp += ystep;
+      if (r + p.dil >= nr) break;
+      U(r + p.dil, ua);
+      out(yp, ub, uc, ud, ua);
+      yp += ystep;
+      if (r + 2 * p.dil >= nr) break;
+      U(r + 2 * p.dil, ub);
+      out(yp, uc, ud, ua, ub);
+      yp += ystep;
+      if (r + 3 * p.dil >= nr) break;
+      U(r + 3 * p.dil, uc);
+      out(yp, ud, ua, ub, uc);
+      yp += ystep;
     }
   }
 }
@@ -469,6 +584,14 @@ cudaError_t launch_gate(const GateParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+namespace {
+constexpr int kRun = 8;
+bool tile_form(const ConvParams& p) {
+  return p.K == 4 && p.conv_w != nullptr && p.dtype == ENGRAM_BF16 && p.H % kTileC == 0 &&
+         p.dil <= kTileMaxDil && p.T >= 2 * kRun * p.dil;
+}
+}  // namespace
+
 cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
   if (p.B <= 0 || p.T <= 0) return cudaSuccess;
   if (p.H % 8 != 0) return cudaErrorInvalidValue;
@@ -476,8 +599,23 @@ cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
   const int64_t blocks = (threads + kConvThreads - 1) / kConvThreads;
   if (blocks > INT32_MAX) return cudaErrorInvalidValue;
   const unsigned nb = static_cast<unsigned>(blocks);
-  constexpr int kRun = 8;
-  if (p.K == 4 && p.conv_w != nullptr && p.T >= 2 * kRun * p.dil) {
+  if (tile_form(p)) {
+    const int64_t tiles = static_cast<int64_t>(p.B) * ((p.T + kTileT - 1) / kTileT);
+    if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+    const int nr = kTileT + 3 * p.dil;
+    const size_t smem = static_cast<size_t>(nr) * kTileC * 2 + static_cast<size_t>(nr) * p.hc * sizeof(float);
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+      const int max_smem = (kTileT + 3 * kTileMaxDil) * (kTileC * 2 + ENGRAM_MAX_HC * 4);
+      cudaError_t e = cudaFuncSetAttribute(conv_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+    launch_k(conv_tile_kernel, dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(p.H / kTileC)),
+             dim3(32 * p.hc), smem, s, p);
+  } else if (p.K == 4 && p.conv_w != nullptr && p.T >= 2 * kRun * p.dil) {
     // run form along each residue class mod dil (the pages' kernel of 4 taps);
     // short chunks (decode) take the flat form below, which shares the taps'
     // loads across the branches
@@ -487,8 +625,14 @@ cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
     const int64_t rb = (nthreads + kConvThreads - 1) / kConvThreads;
     if (rb * kConvThreads > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit thread ids
     const unsigned g = static_cast<unsigned>(rb);
-    if (p.dtype == ENGRAM_F32) launch_k(conv_run_kernel<float, kRun>, dim3(g), dim3(kConvThreads), 0, s, p);
-    else launch_k(conv_run_kernel<uint16_t, kRun>, dim3(g), dim3(kConvThreads), 0, s, p);
+    ConvParams q = p;
+    const uint32_t per_run = static_cast<uint32_t>(p.hc * (p.H / 8));
+    q.div_cg = make_fastdiv(static_cast<uint32_t>(p.H / 8));
+    q.div_run = make_fastdiv(per_run);
+    q.div_cls = make_fastdiv(static_cast<uint32_t>(rpc) * per_run);
+    q.div_b = make_fastdiv(static_cast<uint32_t>(p.dil) * static_cast<uint32_t>(rpc) * per_run);
+    if (p.dtype == ENGRAM_F32) launch_k(conv_run_kernel<float, kRun>, dim3(g), dim3(kConvThreads), 0, s, q);
+    else launch_k(conv_run_kernel<uint16_t, kRun>, dim3(g), dim3(kConvThreads), 0, s, q);
   } else if (p.K <= 4 && p.hc <= 4) {  // up to 4 taps and 4 branches
     if (p.dtype == ENGRAM_F32) launch_k(gated_conv_kernel<float, 4, 4>, dim3(nb), dim3(kConvThreads), 0, s, p);
     else launch_k(gated_conv_kernel<uint16_t, 4, 4>, dim3(nb), dim3(kConvThreads), 0, s, p);

@@ -113,7 +113,7 @@ typedef struct {
  * Initialise with engram_state_init; pass the same state to consecutive calls. */
 typedef struct {
   int64_t* id_ring;  /* DEVICE [B, max_order-1]: last compressed ids, most recent last */
-  void* v_ring;      /* DEVICE [B, ring_len, H] (dtype): V of recent positions, slot = pos % ring_len */
+  void* v_ring;      /* DEVICE [B, ring_len, H] (dtype), 16-byte aligned: V of recent positions, slot = pos % ring_len */
   float* g_ring;     /* DEVICE [B, ring_len, hc]: gates of recent positions */
   int64_t* pos;      /* DEVICE [B]: tokens consumed so far per sequence */
   int32_t ring_len;  /* >= (K-1)*dilation + 1 */

@@ -56,7 +56,7 @@ def test_decode_workload_matches_oracle_and_prefill():
     assert torch.equal(state.id_ring, p.ids[:, S - (w.max_n - 1):])
 
 
-@pytest.mark.parametrize("chunks", [(5, 1, 13, 2, 40), (64,), (1,) * 9 + (55,)])
+@pytest.mark.parametrize("chunks", [(5, 1, 13, 2, 40), (64,), (1,) * 9 + (55,), (10, 70, 64)])
 def test_chunked_prefill_with_state(chunks):
     w = W.small_workload(B=3, T=sum(chunks), orders=(2, 3, 4), dilation=4, hidden=256, hc_mult=2)
     p = device_params(w)
