@@ -580,7 +580,8 @@ int grid_cap() { return num_sms() * 8; }
 cudaError_t launch_gate(const GateParams& p, cudaStream_t s) {
   const int64_t n = p.M * p.hc;
   if (n <= 0) return cudaSuccess;
-  launch_k(gate_kernel, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0, s, p);
+  // small blocks: the few gates of a step spread over every SM
+  launch_k(gate_kernel, dim3(static_cast<unsigned>((n + 63) / 64)), dim3(64), 0, s, p);
   return cudaGetLastError();
 }
 
