@@ -508,6 +508,7 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   hp.raw_vocab = wts->raw_vocab;
   hp.history = state != nullptr ? state->id_ring : nullptr;
   hp.id_ring_out = state != nullptr ? state->id_ring : nullptr;
+  hp.pos_advance = state != nullptr ? state->pos : nullptr;
   hp.rows_out = fused ? rows : nullptr;
   hp.idx_out = nullptr;
   hp.ld_rows = ld;
@@ -550,8 +551,6 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   pp.hc = cfg->hc_mult;
   pp.dtype = cfg->dtype;
   float* g = reinterpret_cast<float*>(w + L.st.g_off);
-  st = run_stage(cfg, pp, g, nullptr, s);
-  if (st != ENGRAM_OK) return st;
 
   // a8-a9: gated value, short conv, residual
   ConvParams cp;
@@ -564,6 +563,7 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
     cp.v_ring = state->v_ring;
     cp.g_ring = state->g_ring;
     cp.pos = state->pos;
+    cp.pos_lag = T;  // advanced next to the id ring update
     cp.ring_len = state->ring_len;
   }
   cp.B = B;
@@ -573,10 +573,12 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   cp.K = cfg->conv_kernel;
   cp.dil = cfg->dilation;
   cp.dtype = cfg->dtype;
+  st = run_stage(cfg, pp, g, nullptr, s);
+  if (st != ENGRAM_OK) return st;
   record(g_events.before_conv, s);
   st = cuda_check(launch_gated_conv(cp, s), "gated conv");
   record(g_events.after_conv, s);
-  if (st != ENGRAM_OK || state == nullptr) return st;
+  if (st != ENGRAM_OK || state == nullptr || conv_writes_rings(cp)) return st;
 
   StateAdvanceParams ap;
   ap.V = pp.V;

@@ -23,6 +23,7 @@ struct HashParams {
   int64_t* idx_out;         // [B*T, nh] int64 or null
   int32_t* rows_out;        // [nh, ld_rows] absolute table rows (int32) or null
   int64_t* id_ring_out;     // decode: [B, n_hist] ring written after use, or null
+  int64_t* pos_advance;     // streaming state: pos [B] += T next to the ring update, or null
   uint32_t* status;
   int64_t raw_vocab;
   int64_t vocab;
@@ -143,10 +144,14 @@ struct ConvParams {
   int32_t ring_len;
   int32_t B, T, H, hc, K, dil;
   engram_dtype dtype;
+  int32_t pos_lag;          // pos [B] already counts this many tokens of the chunk
   // thread decode of the run form (set by launch_gated_conv)
   FastDiv div_b, div_cls, div_run, div_cg;
 };
 cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s);
+// True when launch_gated_conv also writes the chunk's V/g rows into the state
+// rings (one decode step, T == 1), so no state advance follows.
+bool conv_writes_rings(const ConvParams& p);
 
 // Standalone short conv over a materialised u (engram_short_conv).
 struct ShortConvParams {
@@ -159,7 +164,8 @@ struct ShortConvParams {
 };
 cudaError_t launch_short_conv(const ShortConvParams& p, cudaStream_t s);
 
-// Streaming state: write this chunk's last V/g rows into the rings, advance pos.
+// Streaming state: write this chunk's last V/g rows into the rings (pos [B]
+// has already been advanced by T, next to the id ring update).
 struct StateAdvanceParams {
   const void* V;            // [B*T, H]
   const float* g;           // [B*T, hc]
@@ -270,6 +276,16 @@ __device__ __forceinline__ float gate_from_score(float s, float gate_eps) {
   return 1.f / (1.f + expf(-z));
 }
 
+// Gate from the summed score partials of one (token, branch).
+__device__ __forceinline__ float gate_from_sums(float dot, float ssk, float ssq, int H, float rms_eps,
+                                                float gate_eps) {
+  const float invH = 1.f / static_cast<float>(H);
+  const float rk = sqrtf(ssk * invH + rms_eps);
+  const float rq = sqrtf(ssq * invH + rms_eps);
+  const float s = dot / (rk * rq * sqrtf(static_cast<float>(H)));
+  return gate_from_score(s, gate_eps);
+}
+
 // Gate of one (token, branch) from its n_tiles score partials
 // (sum K*nk*nq*Q, sum K^2, sum Q^2 per column tile), summed in tile order:
 //   s = dot / (sqrt(ssk/H + eps) sqrt(ssq/H + eps) sqrt(H)),  g = gate(s).
@@ -290,11 +306,7 @@ __device__ __forceinline__ float gate_from_partials(const float4* part, int n_ti
     ssk += v.y;
     ssq += v.z;
   }
-  const float invH = 1.f / static_cast<float>(H);
-  const float rk = sqrtf(ssk * invH + rms_eps);
-  const float rq = sqrtf(ssq * invH + rms_eps);
-  const float s = dot / (rk * rq * sqrtf(static_cast<float>(H)));
-  return gate_from_score(s, gate_eps);
+  return gate_from_sums(dot, ssk, ssq, H, rms_eps, gate_eps);
 }
 
 }  // namespace engram

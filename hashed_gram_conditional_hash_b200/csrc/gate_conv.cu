@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kConvThreads) gated_conv_kernel(const __grid_c
   const T* vr = static_cast<const T*>(p.v_ring);
   T* Y = static_cast<T*>(p.Y);
   const int K = (W != nullptr) ? p.K : 1;                     // no conv: only U(t)
-  const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) : 0;
+  const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) - p.pos_lag : 0;
 
   // the position itself
   float vt[8], gt[HCMAX];
@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
       gw[k] = __ldg(gp + k * gs);
     }
   } else {
-    const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) : 0;
+    const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) - p.pos_lag : 0;
 #pragma unroll
     for (int k = 0; k < NW; ++k) {
       const int tp = t0 + k * p.dil;
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_tile_kernel(const __g
   const uint16_t* V = static_cast<const uint16_t*>(p.V);
   const uint16_t* vr = static_cast<const uint16_t*>(p.v_ring);
   const int64_t seq = static_cast<int64_t>(b) * p.T;
-  const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) : 0;
+  const int64_t P = (p.pos != nullptr) ? __ldg(p.pos + b) - p.pos_lag : 0;
   const uint32_t sV = static_cast<uint32_t>(__cvta_generic_to_shared(conv_smem));
   float* sG = reinterpret_cast<float*>(conv_smem + static_cast<size_t>(nr) * (kTileC * 2));
 
@@ -487,6 +487,88 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_tile_kernel(const __g
   }
 }
 
+// One decode step (T = 1) with the streaming state, K = 4 taps, bfloat16,
+// 256-channel slices: block (sequence b, slice), one warp per branch, 8
+// channels per lane.  Thread 0 turns pos into the ring rows of the taps at
+// t - 3 dil, t - 2 dil, t - dil (the ring holds (K-1) dil + 1 >= 3 dil + 1
+// positions, slot = position mod ring length); then every lane loads its
+// 16-byte pieces of V(t) and of those three ring rows, the four gates and its
+// taps, and stores 8 channels of Y.  The same kernel is the step's state
+// advance: the branch-0 warp writes V(t) and lanes 0 write g(t) into t's
+// slot, which no tap of this step reads.
+__global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __grid_constant__ ConvParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  constexpr int K = 4;
+  __shared__ int64_t s_row[K];   // ring row (b * ring_len + slot) of tap i; -1 before the start
+  const int b = static_cast<int>(blockIdx.x);
+  const int tid = static_cast<int>(threadIdx.x);
+  const int h = tid >> 5, lane = tid & 31;
+  const bool worker = h < p.hc;
+  const int c = static_cast<int>(blockIdx.y) * kTileC + lane * 8;
+  const uint16_t* V = static_cast<const uint16_t*>(p.V);
+  uint16_t* vr = static_cast<uint16_t*>(const_cast<void*>(p.v_ring));
+  float* gr = const_cast<float*>(p.g_ring);
+  if (tid == 0) {
+    const int64_t P = __ldg(p.pos + b) - p.pos_lag;   // position of this step's token
+    const int64_t slot_t = P % p.ring_len;
+#pragma unroll
+    for (int i = 0; i < K; ++i) {                     // tap i sits at t - (K-1-i) dil
+      const int64_t back = static_cast<int64_t>(K - 1 - i) * p.dil;
+      int64_t slot = slot_t - back;
+      if (slot < 0) slot += p.ring_len;
+      s_row[i] = (P - back >= 0) ? static_cast<int64_t>(b) * p.ring_len + slot : -1;
+    }
+  }
+  __syncthreads();
+  if (!worker) return;
+  uint4 raw[K];
+  float gg[K];
+#pragma unroll
+  for (int i = 0; i < K - 1; ++i) {
+    const int64_t row = s_row[i];
+    if (row >= 0) {
+      raw[i] = __ldg(reinterpret_cast<const uint4*>(vr + row * p.H + c));
+      gg[i] = __ldg(gr + row * p.hc + h);
+    } else {
+      raw[i] = make_uint4(0, 0, 0, 0);
+      gg[i] = 0.f;
+    }
+  }
+  raw[K - 1] = __ldg(reinterpret_cast<const uint4*>(V + static_cast<int64_t>(b) * p.H + c));
+  gg[K - 1] = __ldg(p.g + static_cast<int64_t>(b) * p.hc + h);
+  float2 w2[4][K];                                // [channel pair][tap]
+  {
+    float w[8][K];
+    load_taps<uint16_t, K>(static_cast<const uint16_t*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, K, w);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < K; ++i) w2[j][i] = make_float2(w[2 * j][i], w[2 * j + 1][i]);
+  }
+  float2 u[K][4];
+#pragma unroll
+  for (int i = 0; i < K; ++i) {
+    float2 v[4];
+    Pair8<uint16_t>::unpack(raw[i], v);
+    const float2 g2 = make_float2(gg[i], gg[i]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) u[i][j] = __fmul2_rn(g2, v[j]);
+  }
+  float2 acc[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float2 a = u[K - 1][j];
+#pragma unroll
+    for (int i = 0; i < K; ++i) a = __ffma2_rn(w2[j][i], u[i][j], a);
+    acc[j] = a;
+  }
+  Pair8<uint16_t>::store(static_cast<uint16_t*>(p.Y) + (static_cast<int64_t>(b) * p.hc + h) * p.H + c, acc);
+  // the step's state advance
+  const int64_t row_t = s_row[K - 1];
+  if (h == 0) *reinterpret_cast<uint4*>(vr + row_t * p.H + c) = raw[K - 1];
+  if (blockIdx.y == 0 && lane == 0) gr[row_t * p.hc + h] = gg[K - 1];
+}
+
 // -------------------------------------------------------------- standalone conv
 template <typename T>
 __global__ void short_conv_kernel(const __grid_constant__ ShortConvParams p) {
@@ -541,7 +623,7 @@ template <typename T>
 __global__ void state_advance_kernel(const __grid_constant__ StateAdvanceParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int b = blockIdx.x;
-  const int64_t P = p.pos[b];
+  const int64_t P = p.pos[b] - p.T;   // position of the chunk's first token
   const int n = min(p.T, p.ring_len);
   const T* V = static_cast<const T*>(p.V);
   T* vr = static_cast<T*>(p.v_ring);
@@ -553,8 +635,6 @@ __global__ void state_advance_kernel(const __grid_constant__ StateAdvanceParams 
     for (int c = threadIdx.x; c < p.H; c += blockDim.x) vr[dst * p.H + c] = V[src * p.H + c];
     for (int h = threadIdx.x; h < p.hc; h += blockDim.x) p.g_ring[dst * p.hc + h] = p.g[src * p.hc + h];
   }
-  __syncthreads();
-  if (threadIdx.x == 0) p.pos[b] = P + p.T;
 }
 
 __global__ void state_init_kernel(int64_t* id_ring, int n_hist, uint16_t* v_ring16, float* v_ring32,
@@ -593,9 +673,19 @@ bool tile_form(const ConvParams& p) {
 }
 }  // namespace
 
+bool conv_writes_rings(const ConvParams& p) {
+  return p.T == 1 && p.pos != nullptr && p.v_ring != nullptr && p.g_ring != nullptr && p.K == 4 &&
+         p.conv_w != nullptr && p.dtype == ENGRAM_BF16 && p.H % kTileC == 0 && p.hc <= ENGRAM_MAX_HC;
+}
+
 cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
   if (p.B <= 0 || p.T <= 0) return cudaSuccess;
   if (p.H % 8 != 0) return cudaErrorInvalidValue;
+  if (conv_writes_rings(p)) {
+    launch_k(conv_step_kernel, dim3(static_cast<unsigned>(p.B), static_cast<unsigned>(p.H / kTileC)),
+             dim3(32 * p.hc), 0, s, p);
+    return cudaGetLastError();
+  }
   const int64_t threads = static_cast<int64_t>(p.B) * p.T * (p.H / 8);
   const int64_t blocks = (threads + kConvThreads - 1) / kConvThreads;
   if (blocks > INT32_MAX) return cudaErrorInvalidValue;

@@ -104,16 +104,20 @@ __global__ void id_ring_kernel(const __grid_constant__ HashParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= p.B) return;
-  int64_t* ring = p.id_ring_out + static_cast<int64_t>(b) * p.n_hist;
-  const int64_t base = static_cast<int64_t>(b) * p.T;
-  // ascending j reads index j + T >= j before writing j (in-place forward shift)
-  for (int j = 0; j < p.n_hist; ++j) {
-    int src = j + p.T;  // position in (old ring ++ chunk)
-    int64_t v;
-    if (src < p.n_hist) v = ring[src];
-    else v = load_id(p, __ldg(p.ids + base + (src - p.n_hist)));
-    ring[j] = v;
+  if (p.id_ring_out != nullptr) {
+    int64_t* ring = p.id_ring_out + static_cast<int64_t>(b) * p.n_hist;
+    const int64_t base = static_cast<int64_t>(b) * p.T;
+    // ascending j reads index j + T >= j before writing j (in-place forward shift)
+    for (int j = 0; j < p.n_hist; ++j) {
+      int src = j + p.T;  // position in (old ring ++ chunk)
+      int64_t v;
+      if (src < p.n_hist) v = ring[src];
+      else v = load_id(p, __ldg(p.ids + base + (src - p.n_hist)));
+      ring[j] = v;
+    }
   }
+  // the sequence has consumed this chunk; later kernels of the call read pos - T
+  if (p.pos_advance != nullptr) p.pos_advance[b] += p.T;
 }
 
 // Id at position t of sequence b (pad / history before the start), compressed
@@ -207,7 +211,7 @@ cudaError_t launch_hash(const HashParams& p, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (p.id_ring_out != nullptr && p.n_hist > 0 && p.B > 0) {
+  if (((p.id_ring_out != nullptr && p.n_hist > 0) || p.pos_advance != nullptr) && p.B > 0) {
     launch_k(id_ring_kernel, dim3((p.B + 127) / 128), dim3(128), 0, s, p);
     return cudaGetLastError();
   }
@@ -224,7 +228,7 @@ cudaError_t launch_hash_gather(const HashGatherParams& g, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (p.id_ring_out != nullptr && p.n_hist > 0 && p.B > 0) {
+  if (((p.id_ring_out != nullptr && p.n_hist > 0) || p.pos_advance != nullptr) && p.B > 0) {
     launch_k(id_ring_kernel, dim3((p.B + 127) / 128), dim3(128), 0, s, p);
     return cudaGetLastError();
   }
