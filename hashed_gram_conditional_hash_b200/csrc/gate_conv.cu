@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
 }
 
 // Tile form for K = 4 taps, bfloat16, 256-channel slices.  A block owns
-// kTileT consecutive positions of one sequence and one 256-channel slice, all
+// kTileT (48) consecutive positions of one sequence and one 256-channel slice, all
 // branches (one warp per branch, 8 channels per lane).  It first copies the V
 // rows of the tile and of its 3*dil-row halo into shared memory with cp.async
 // (one 16-byte piece per request, no registers held; halo rows before the
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
 // 16-byte shared load, 8 channels of U, 4 taps two channels per instruction
 // (__ffma2_rn), one coalesced 16-byte store of Y.  Global memory sees each V
 // row once per tile (plus the halo) and each Y element once.
-constexpr int kTileT = 32;        // positions per block
+constexpr int kTileT = 48;        // positions per block
 constexpr int kTileC = 256;       // channels per block (512 bytes of a bf16 row)
 constexpr int kTileMaxDil = 32;   // longer halos take the run form
 

@@ -135,36 +135,61 @@ __device__ __forceinline__ uint64_t token_at(const HashParams& p, int b, int t) 
   return static_cast<uint64_t>(p.pad_id);
 }
 
-// One warp produces 32 consecutive rows of e (row q = m*nh + h): lane l
-// hashes row q0 + l (its order's window read through L1, xor of products,
-// Barrett reduction by its head's prime), then the warp copies the 32 table
-// rows with every 16-byte load issued before the stores.
+// Absolute table row of row q = m*nh + h of e: the window of token m's order
+// (read through L1), xor of the products, Barrett reduction by head h's prime.
+__device__ __forceinline__ int64_t hashed_row(const HashParams& p, int q) {
+  const int m = q / p.nh;
+  const int h = q - m * p.nh;
+  const int o = h / p.J;
+  const int b = m / p.T;
+  const int t = m - b * p.T;
+  const int n = p.orders[o];
+  uint64_t mix = token_at(p, b, t) * p.mult[0];
+#pragma unroll
+  for (int k = 1; k < ENGRAM_MAX_NGRAM; ++k)
+    if (k < n) mix ^= token_at(p, b, t - k) * p.mult[k];
+  return p.row_off[h] + static_cast<int64_t>(barrett_mod(mix, p.prime[h], p.barrett[h]));
+}
+
+// One warp produces ROWS (16 or 32) consecutive rows of e (row q = m*nh + h):
+// lane l < ROWS hashes row l, then the warp copies the table rows with every
+// 16-byte load issued before the stores.  CH = 16-byte pieces per row when
+// known at compile time (8: 64 bf16), else 0 (read from the params; ROWS 32).
+// Fewer rows per warp means more warps, each with one short dependent chain
+// (ids -> hash -> rows -> e), which is what the random row reads want.
+template <int CH, int ROWS>
 __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant__ HashGatherParams g) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const HashParams& p = g.h;
   const int lane = threadIdx.x & 31;
   // rows of e (B*T*nh) stay below 2^31 (checked by the launcher): 32-bit math
   const int total = p.B * p.T * p.nh;
-  const int q0 = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x) - lane;
+  const int q0 = ((static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x)) >> 5) * ROWS;
   if (q0 >= total) return;
-  const int q = q0 + lane;
-  int64_t row = 0;
-  if (q < total) {
-    const int m = q / p.nh;
-    const int h = q - m * p.nh;
-    const int o = h / p.J;
-    const int b = m / p.T;
-    const int t = m - b * p.T;
-    const int n = p.orders[o];
-    uint64_t mix = token_at(p, b, t) * p.mult[0];
+  const int q = q0 + (lane % ROWS);
+  const int64_t row = q < total ? hashed_row(p, q) : 0;
+  const char* tab = static_cast<const char*>(g.table);
+  if (CH > 0) {
+    // piece i of the warp's rows is row i / CH, 16-byte column i % CH
+    constexpr int kPer = ROWS * (CH > 0 ? CH : 1) / 32;   // pieces per lane
+    int4 v[kPer];
 #pragma unroll
-    for (int k = 1; k < ENGRAM_MAX_NGRAM; ++k)
-      if (k < n) mix ^= token_at(p, b, t - k) * p.mult[k];
-    row = p.row_off[h] + static_cast<int64_t>(barrett_mod(mix, p.prime[h], p.barrett[h]));
+    for (int u = 0; u < kPer; ++u) {
+      const int i = u * 32 + lane;
+      const int r = i / CH;
+      const int64_t src = __shfl_sync(0xffffffffu, row, r);
+      if (q0 + r < total) v[u] = __ldg(reinterpret_cast<const int4*>(tab + src * (CH * 16)) + (i - r * CH));
+    }
+    int4* out = static_cast<int4*>(g.e) + static_cast<int64_t>(q0) * CH;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = u * 32 + lane;
+      if (q0 + i / CH < total) out[i] = v[u];
+    }
+    return;
   }
   const int chunks = g.row_bytes >> 4;          // 16-byte chunks per row
-  const int per = 32 * chunks;                   // chunks of this warp's 32 rows
-  const char* tab = static_cast<const char*>(g.table);
+  const int per = ROWS * chunks;                 // chunks of the warp's rows
   int4* out = static_cast<int4*>(g.e) + static_cast<int64_t>(q0) * chunks;
   constexpr int kBatch = 8;
   for (int base = 0; base < per; base += 32 * kBatch) {
@@ -173,7 +198,7 @@ __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant_
     for (int u = 0; u < kBatch; ++u) {
       const int i = base + u * 32 + lane;
       const int r = i / chunks;
-      const int64_t src = __shfl_sync(0xffffffffu, row, r & 31);
+      const int64_t src = __shfl_sync(0xffffffffu, row, r % ROWS);
       if (i < per && q0 + r < total)
         v[u] = __ldg(reinterpret_cast<const int4*>(tab + src * g.row_bytes) + (i - r * chunks));
     }
@@ -222,9 +247,15 @@ cudaError_t launch_hash_gather(const HashGatherParams& g, cudaStream_t s) {
   const HashParams& p = g.h;
   const int64_t total = static_cast<int64_t>(p.B) * p.T * p.nh;
   if (total > 0) {
-    const int64_t blocks = (total + 255) / 256;
-    if (blocks * 256 > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit row ids in the kernel
-    launch_k(hash_gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
+    constexpr int kRows = 16;                    // rows per warp for 128-byte rows
+    if (total * (32 / kRows) + 256 > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit ids in the kernel
+    if (g.row_bytes == 128) {
+      const int64_t blocks = (total + 8 * kRows - 1) / (8 * kRows);
+      launch_k(hash_gather_kernel<8, kRows>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
+    } else {
+      const int64_t blocks = (total + 255) / 256;
+      launch_k(hash_gather_kernel<0, 32>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
