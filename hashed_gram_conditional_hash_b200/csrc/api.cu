@@ -170,10 +170,12 @@ engram_status run_projection(const engram_config* c, ProjParams* pp, cudaStream_
 
 // Projection followed by the stand-alone gate kernel (engram_gate_fuse).
 engram_status run_stage(const engram_config* c, ProjParams pp, float* g, float* g_copy,
-                        cudaStream_t s) {
+                        cudaStream_t s, const StateIdsAdvance* state_ids = nullptr) {
   engram_status st = run_projection(c, &pp, s);
   if (st != ENGRAM_OK) return st;
   GateParams gp;
+  memset(&gp, 0, sizeof gp);
+  if (state_ids != nullptr) gp.state = *state_ids;
   gp.partials = pp.partials;
   gp.g = g;
   gp.g_copy = g_copy;
@@ -507,8 +509,6 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   hp.lookup = wts->lookup;
   hp.raw_vocab = wts->raw_vocab;
   hp.history = state != nullptr ? state->id_ring : nullptr;
-  hp.id_ring_out = state != nullptr ? state->id_ring : nullptr;
-  hp.pos_advance = state != nullptr ? state->pos : nullptr;
   hp.rows_out = fused ? rows : nullptr;
   hp.idx_out = nullptr;
   hp.ld_rows = ld;
@@ -563,7 +563,7 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
     cp.v_ring = state->v_ring;
     cp.g_ring = state->g_ring;
     cp.pos = state->pos;
-    cp.pos_lag = T;  // advanced next to the id ring update
+    cp.pos_lag = T;  // advanced by the gate kernel
     cp.ring_len = state->ring_len;
   }
   cp.B = B;
@@ -573,7 +573,24 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   cp.K = cfg->conv_kernel;
   cp.dil = cfg->dilation;
   cp.dtype = cfg->dtype;
-  st = run_stage(cfg, pp, g, nullptr, s);
+  // with the streaming state the gate kernel also takes the chunk's ids into
+  // the id ring (the hash has read it) and advances pos (the conv reads pos - T)
+  StateIdsAdvance sa;
+  memset(&sa, 0, sizeof sa);
+  if (state != nullptr) {
+    sa.id_ring = state->id_ring;
+    sa.pos = state->pos;
+    sa.ids = ids;
+    sa.lookup = wts->lookup;
+    sa.status = dev_status;
+    sa.raw_vocab = wts->raw_vocab;
+    sa.vocab = cfg->vocab;
+    sa.pad_id = cfg->pad_id;
+    sa.B = B;
+    sa.T = T;
+    sa.n_hist = hp.n_hist;
+  }
+  st = run_stage(cfg, pp, g, nullptr, s, state != nullptr ? &sa : nullptr);
   if (st != ENGRAM_OK) return st;
   record(g_events.before_conv, s);
   st = cuda_check(launch_gated_conv(cp, s), "gated conv");

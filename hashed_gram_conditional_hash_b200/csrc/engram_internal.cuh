@@ -13,6 +13,26 @@ namespace engram {
 
 // ---------------------------------------------------------------- host side
 
+// Division of a non-negative 32-bit integer n < 2^31 by a divisor d fixed
+// at launch: q = (umulhi(n, mul) + n) >> shift, with shift = ceil(log2 d)
+// and mul = floor(2^32 (2^shift - d) / d) + 1 (the invariant-divisor method
+// of Granlund and Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994).  umulhi(n, mul) < n keeps the sum below 2^32.
+struct FastDiv {
+  uint32_t d = 1, mul = 1, shift = 0;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.shift = 0;
+  while ((static_cast<uint64_t>(1) << f.shift) < d) ++f.shift;
+  f.mul = static_cast<uint32_t>(((static_cast<uint64_t>(1) << 32) * ((static_cast<uint64_t>(1) << f.shift) - d)) / d + 1);
+  return f;
+}
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
+  return (__umulhi(n, f.mul) + n) >> f.shift;
+}
+
 // Per-call parameters of the hash kernel (a1-a3).  The small per-head arrays
 // travel in the kernel's parameter space, so every thread reads them from the
 // constant bank.
@@ -22,8 +42,6 @@ struct HashParams {
   const int64_t* history;   // [B, n_hist] or null (then pad_id)
   int64_t* idx_out;         // [B*T, nh] int64 or null
   int32_t* rows_out;        // [nh, ld_rows] absolute table rows (int32) or null
-  int64_t* id_ring_out;     // decode: [B, n_hist] ring written after use, or null
-  int64_t* pos_advance;     // streaming state: pos [B] += T next to the ring update, or null
   uint32_t* status;
   int64_t raw_vocab;
   int64_t vocab;
@@ -48,6 +66,7 @@ struct HashGatherParams {
   const void* table;
   void* e;                  // [B*T, nh*Dh]
   int32_t row_bytes;
+  FastDiv div_nh, div_J, div_T;   // set by launch_hash_gather
 };
 cudaError_t launch_hash_gather(const HashGatherParams& p, cudaStream_t s);
 
@@ -99,6 +118,19 @@ cudaError_t launch_proj_tc(const ProjParams& p, cudaStream_t s);
 cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s);
 
 // Gate finalisation (a6 reduction + a7): g[m, h] from the partials.
+// The streaming state's id bookkeeping of one chunk, done by the gate kernel
+// (after the hash has read the ring, before the conv reads pos): the id ring
+// takes the chunk's last ids and pos advances by T.
+struct StateIdsAdvance {
+  int64_t* id_ring;         // [B, n_hist]
+  int64_t* pos;             // [B]; null: nothing to do
+  const int64_t* ids;       // [B, T] chunk ids (raw when lookup != null)
+  const int64_t* lookup;    // [raw_vocab] or null
+  uint32_t* status;
+  int64_t raw_vocab, vocab, pad_id;
+  int32_t B, T, n_hist;
+};
+
 struct GateParams {
   const float4* partials;   // [M, hc, n_tiles]
   float* g;                 // [M, hc]
@@ -106,28 +138,9 @@ struct GateParams {
   int64_t M;
   int32_t hc, n_tiles, H;
   float rms_eps, gate_eps;
+  StateIdsAdvance state;    // state.pos == null: no streaming state
 };
 cudaError_t launch_gate(const GateParams& p, cudaStream_t s);
-
-// Division of a non-negative 32-bit integer n < 2^31 by a divisor d fixed
-// at launch: q = (umulhi(n, mul) + n) >> shift, with shift = ceil(log2 d)
-// and mul = floor(2^32 (2^shift - d) / d) + 1 (the invariant-divisor method
-// of Granlund and Montgomery, "Division by invariant integers using
-// multiplication", PLDI 1994).  umulhi(n, mul) < n keeps the sum below 2^32.
-struct FastDiv {
-  uint32_t d = 1, mul = 1, shift = 0;
-};
-inline FastDiv make_fastdiv(uint32_t d) {
-  FastDiv f;
-  f.d = d;
-  f.shift = 0;
-  while ((static_cast<uint64_t>(1) << f.shift) < d) ++f.shift;
-  f.mul = static_cast<uint32_t>(((static_cast<uint64_t>(1) << 32) * ((static_cast<uint64_t>(1) << f.shift) - d)) / d + 1);
-  return f;
-}
-__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f) {
-  return (__umulhi(n, f.mul) + n) >> f.shift;
-}
 
 // Gated value + short conv + residual (a8, a9) from V and the gates.
 //   Y[b,t,h,c] = U(t) + sum_i w[h*H+c, i] U(t - (K-1-i) dil),  U(t) = g[t,h] V[t,c]
@@ -145,6 +158,7 @@ struct ConvParams {
   int32_t B, T, H, hc, K, dil;
   engram_dtype dtype;
   int32_t pos_lag;          // pos [B] already counts this many tokens of the chunk
+  int32_t tile_t;           // positions per block of the tile form (set by launch_gated_conv)
   // thread decode of the run form (set by launch_gated_conv)
   FastDiv div_b, div_cls, div_run, div_cg;
 };
@@ -165,7 +179,7 @@ struct ShortConvParams {
 cudaError_t launch_short_conv(const ShortConvParams& p, cudaStream_t s);
 
 // Streaming state: write this chunk's last V/g rows into the rings (pos [B]
-// has already been advanced by T, next to the id ring update).
+// has already been advanced by T, by the gate kernel).
 struct StateAdvanceParams {
   const void* V;            // [B*T, H]
   const float* g;           // [B*T, hc]
@@ -255,6 +269,26 @@ template <> struct Elem<uint16_t> {
     p[i] = f32_to_bf16(v);
   }
 };
+
+// Compressed id of a raw id (lookup != null) or a compressed id checked
+// against [0, vocab); out-of-range ids set ENGRAM_STATUS_ID_RANGE and become
+// pad_id.
+__device__ __forceinline__ int64_t checked_id(int64_t raw, const int64_t* lookup, int64_t raw_vocab, int64_t vocab,
+                                              int64_t pad_id, uint32_t* status) {
+  int64_t x = raw;
+  if (lookup != nullptr) {
+    if (raw < 0 || raw >= raw_vocab) {
+      set_status(status, ENGRAM_STATUS_ID_RANGE);
+      return pad_id;
+    }
+    x = __ldg(lookup + raw);
+  }
+  if (x < 0 || x >= vocab) {
+    set_status(status, ENGRAM_STATUS_ID_RANGE);
+    return pad_id;
+  }
+  return x;
+}
 
 // Exact x mod p for x < 2^64, p >= 2, with mu = floor((2^64 - 1) / p)
 // (Barrett reduction: the estimate q = floor(x * mu / 2^64) never exceeds

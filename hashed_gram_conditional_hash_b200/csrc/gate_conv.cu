@@ -22,6 +22,22 @@ namespace {
 __global__ void gate_kernel(const __grid_constant__ GateParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  const StateIdsAdvance& st = p.state;
+  if (st.pos != nullptr && i < st.B) {
+    // the streaming state's ids (M*hc >= B threads): the ring becomes the last
+    // n_hist ids of (old ring ++ chunk), ascending j reading index j + T >= j
+    // before it is overwritten; pos advances by T
+    const int b = static_cast<int>(i);
+    int64_t* ring = st.id_ring + static_cast<int64_t>(b) * st.n_hist;
+    const int64_t base = static_cast<int64_t>(b) * st.T;
+    for (int j = 0; j < st.n_hist; ++j) {
+      const int src = j + st.T;               // position in (old ring ++ chunk)
+      ring[j] = src < st.n_hist ? ring[src]
+                                : checked_id(__ldg(st.ids + base + (src - st.n_hist)), st.lookup, st.raw_vocab,
+                                             st.vocab, st.pad_id, st.status);
+    }
+    st.pos[b] += st.T;
+  }
   if (i >= p.M * p.hc) return;
   const float g = gate_from_partials(p.partials + i * p.n_tiles, p.n_tiles, p.H, p.rms_eps, p.gate_eps);
   p.g[i] = g;
@@ -348,7 +364,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
 }
 
 // Tile form for K = 4 taps, bfloat16, 256-channel slices.  A block owns
-// kTileT (48) consecutive positions of one sequence and one 256-channel slice, all
+// tile_t (32 to 64) consecutive positions of one sequence and one 256-channel slice, all
 // branches (one warp per branch, 8 channels per lane).  It first copies the V
 // rows of the tile and of its 3*dil-row halo into shared memory with cp.async
 // (one 16-byte piece per request, no registers held; halo rows before the
@@ -358,7 +374,8 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
 // 16-byte shared load, 8 channels of U, 4 taps two channels per instruction
 // (__ffma2_rn), one coalesced 16-byte store of Y.  Global memory sees each V
 // row once per tile (plus the halo) and each Y element once.
-constexpr int kTileT = 48;        // positions per block
+constexpr int kTileTMin = 32;     // positions per block: the launcher picks one in
+constexpr int kTileTMax = 64;     // [32, 64] that spreads the blocks evenly over the SMs
 constexpr int kTileC = 256;       // channels per block (512 bytes of a bf16 row)
 constexpr int kTileMaxDil = 32;   // longer halos take the run form
 
@@ -369,16 +386,68 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_tile_kernel(const __grid_constant__ ConvParams p) {
+// CPL channels of one row held by a lane as CPL/2 channel pairs: the packed
+// bf16 form in shared memory (16 or 8 bytes), its unpacking, and the store of
+// the lane's CPL outputs.
+template <int CPL> struct LaneRow;
+template <> struct LaneRow<8> {
+  using raw_t = uint4;
+  static __device__ __forceinline__ raw_t lds(uint32_t a) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
+    return r;
+  }
+  static __device__ __forceinline__ void unpack(const raw_t& w, float2 (&v)[4]) { Pair8<uint16_t>::unpack(w, v); }
+  static __device__ __forceinline__ void store(uint16_t* p, const float2 (&v)[4]) { Pair8<uint16_t>::store(p, v); }
+};
+template <> struct LaneRow<4> {
+  using raw_t = uint2;
+  static __device__ __forceinline__ raw_t lds(uint32_t a) {
+    uint2 r;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a));
+    return r;
+  }
+  static __device__ __forceinline__ void unpack(const raw_t& w, float2 (&v)[2]) {
+    v[0] = make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
+    v[1] = make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+  }
+  static __device__ __forceinline__ void store(uint16_t* p, const float2 (&v)[2]) {
+    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0].x, v[0].y), pack_bf16x2(v[1].x, v[1].y));
+  }
+};
+
+// The K = 4 taps of CPL consecutive channels (4*CPL contiguous bf16 values,
+// channel-major) as w2[pair][tap] = (tap of channel 2 pair, of channel 2 pair + 1).
+template <int CPL>
+__device__ __forceinline__ void load_taps_pairs(const uint16_t* row, float2 (&w2)[CPL / 2][4]) {
+  const uint4* q = reinterpret_cast<const uint4*>(row);
+#pragma unroll
+  for (int u = 0; u < CPL / 2; ++u) {        // 8 values = channels 2u, 2u+1, taps 0..3
+    const uint4 x = __ldg(q + u);
+    const uint32_t a[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {            // value 8u + 2e and 8u + 2e + 1
+      const int k0 = 8 * u + 2 * e, k1 = k0 + 1;
+      const float f0 = __uint_as_float(a[e] << 16), f1 = __uint_as_float(a[e] & 0xffff0000u);
+      if ((k0 >> 2) & 1) w2[u][k0 & 3].y = f0; else w2[u][k0 & 3].x = f0;
+      if ((k1 >> 2) & 1) w2[u][k1 & 3].y = f1; else w2[u][k1 & 3].x = f1;
+    }
+  }
+}
+
+template <int CPL>
+__global__ void __launch_bounds__((kTileC / CPL) * ENGRAM_MAX_HC) conv_tile_kernel(const __grid_constant__ ConvParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   constexpr int K = 4;
+  constexpr int LPB = kTileC / CPL;                // lanes (threads) per branch
+  constexpr int NP = CPL / 2;                      // channel pairs per lane
   extern __shared__ __align__(16) uint8_t conv_smem[];
-  const int tiles_per_seq = (p.T + kTileT - 1) / kTileT;
+  const int tiles_per_seq = (p.T + p.tile_t - 1) / p.tile_t;
   const int b = static_cast<int>(blockIdx.x) / tiles_per_seq;
-  const int t0 = (static_cast<int>(blockIdx.x) - b * tiles_per_seq) * kTileT;
+  const int t0 = (static_cast<int>(blockIdx.x) - b * tiles_per_seq) * p.tile_t;
   const int c0 = static_cast<int>(blockIdx.y) * kTileC;
   const int halo = (K - 1) * p.dil;
-  const int n_out = min(kTileT, p.T - t0);
+  const int n_out = min(p.tile_t, p.T - t0);
   const int nr = n_out + halo;                      // smem row r is position t0 - halo + r
   const int nthreads = static_cast<int>(blockDim.x);
   const int tid = static_cast<int>(threadIdx.x);
@@ -417,41 +486,31 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_tile_kernel(const __g
   cp_async_wait_all();
   __syncthreads();
 
-  // ---- one warp per branch, 8 channels per lane
-  const int h = tid >> 5, lane = tid & 31;
+  // ---- LPB threads per branch, CPL channels per thread
+  const int h = tid / LPB, lane = tid - h * LPB;
   if (h >= p.hc) return;
-  const int c = c0 + lane * 8;
-  float2 w2[4][K];                                // [channel pair][tap]
-  {
-    float w[8][K];
-    load_taps<uint16_t, K>(static_cast<const uint16_t*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, K, w);
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int i = 0; i < K; ++i) w2[j][i] = make_float2(w[2 * j][i], w[2 * j + 1][i]);
-  }
-  const uint32_t lane_off = sV + static_cast<uint32_t>(lane * 16);
-  auto U = [&](int r, float2 (&u)[4]) {            // U of smem row r, this lane's channels
-    uint4 raw;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(raw.x), "=r"(raw.y), "=r"(raw.z), "=r"(raw.w)
-                 : "r"(lane_off + static_cast<uint32_t>(r * (kTileC * 2))));
-    float2 v[4];
-    Pair8<uint16_t>::unpack(raw, v);
+  const int c = c0 + lane * CPL;
+  float2 w2[NP][K];                               // [channel pair][tap]
+  load_taps_pairs<CPL>(static_cast<const uint16_t*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, w2);
+  const uint32_t lane_off = sV + static_cast<uint32_t>(lane * CPL * 2);
+  auto U = [&](int r, float2 (&u)[NP]) {           // U of smem row r, this thread's channels
+    const typename LaneRow<CPL>::raw_t raw = LaneRow<CPL>::lds(lane_off + static_cast<uint32_t>(r * (kTileC * 2)));
+    float2 v[NP];
+    LaneRow<CPL>::unpack(raw, v);
     const float gg = sG[r * p.hc + h];
     const float2 g2 = make_float2(gg, gg);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) u[j] = __fmul2_rn(g2, v[j]);
+    for (int j = 0; j < NP; ++j) u[j] = __fmul2_rn(g2, v[j]);
   };
   uint16_t* Y = static_cast<uint16_t*>(p.Y);
   const int64_t ystep = static_cast<int64_t>(p.dil) * p.hc * p.H;
   // output at row r (position t0 - halo + r) from taps in slots A (r - 3 dil),
   // B (r - 2 dil), C (r - dil) and D (r, written here)
-  auto out = [&](uint16_t* yp, const float2 (&A)[4], const float2 (&Bv)[4], const float2 (&C)[4],
-                 const float2 (&D)[4]) {
-    float2 acc[4];
+  auto out = [&](uint16_t* yp, const float2 (&A)[NP], const float2 (&Bv)[NP], const float2 (&C)[NP],
+                 const float2 (&D)[NP]) {
+    float2 acc[NP];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < NP; ++j) {
       float2 a = D[j];
       a = __ffma2_rn(w2[j][0], A[j], a);
       a = __ffma2_rn(w2[j][1], Bv[j], a);
@@ -459,10 +518,10 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_tile_kernel(const __g
       a = __ffma2_rn(w2[j][3], D[j], a);
       acc[j] = a;
     }
-    Pair8<uint16_t>::store(yp, acc);
+    LaneRow<CPL>::store(yp, acc);
   };
   for (int cls = 0; cls < p.dil && cls < n_out; ++cls) {
-    float2 ua[4], ub[4], uc[4], ud[4];
+    float2 ua[NP], ub[NP], uc[NP], ud[NP];
     U(cls, ua);
     U(cls + p.dil, ub);
     U(cls + 2 * p.dil, uc);
@@ -691,21 +750,38 @@ cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
   if (blocks > INT32_MAX) return cudaErrorInvalidValue;
   const unsigned nb = static_cast<unsigned>(blocks);
   if (tile_form(p)) {
-    const int64_t tiles = static_cast<int64_t>(p.B) * ((p.T + kTileT - 1) / kTileT);
-    if (tiles > INT32_MAX) return cudaErrorInvalidValue;
-    const int nr = kTileT + 3 * p.dil;
-    const size_t smem = static_cast<size_t>(nr) * kTileC * 2 + static_cast<size_t>(nr) * p.hc * sizeof(float);
+    constexpr int kCpl = 8;                        // channels per thread (4 was slower)
+    const int threads = (kTileC / kCpl) * p.hc;
+    const int slices = p.H / kTileC;
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-      const int max_smem = (kTileT + 3 * kTileMaxDil) * (kTileC * 2 + ENGRAM_MAX_HC * 4);
-      cudaError_t e = cudaFuncSetAttribute(conv_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+      const int max_smem = (kTileTMax + 3 * kTileMaxDil) * (kTileC * 2 + ENGRAM_MAX_HC * 4);
+      cudaError_t e = cudaFuncSetAttribute(conv_tile_kernel<kCpl>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           max_smem);
       if (e != cudaSuccess) return e;
       attr_set[dev] = true;
     }
-    launch_k(conv_tile_kernel, dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(p.H / kTileC)),
-             dim3(32 * p.hc), smem, s, p);
+    // tile length: the per-SM work ceil(blocks / SMs) * (tile + halo) is
+    // smallest when the blocks spread evenly (model-shaped: 46 tiles of 45)
+    const int sms = num_sms();
+    ConvParams q = p;
+    int64_t best = -1;
+    for (int tt = kTileTMin; tt <= kTileTMax; ++tt) {
+      const int64_t blocks = static_cast<int64_t>(p.B) * ((p.T + tt - 1) / tt) * slices;
+      const int64_t cost = ((blocks + sms - 1) / sms) * (tt + 3 * p.dil);
+      if (best < 0 || cost < best) {
+        best = cost;
+        q.tile_t = tt;
+      }
+    }
+    const int64_t tiles = static_cast<int64_t>(p.B) * ((p.T + q.tile_t - 1) / q.tile_t);
+    if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+    const int nr = q.tile_t + 3 * p.dil;
+    const size_t smem = static_cast<size_t>(nr) * kTileC * 2 + static_cast<size_t>(nr) * p.hc * sizeof(float);
+    launch_k(conv_tile_kernel<kCpl>, dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(slices)),
+             dim3(threads), smem, s, q);
   } else if (p.K == 4 && p.conv_w != nullptr && p.T >= 2 * kRun * p.dil) {
     // run form along each residue class mod dil (the pages' kernel of 4 taps);
     // short chunks (decode) take the flat form below, which shares the taps'

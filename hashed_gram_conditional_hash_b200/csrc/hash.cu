@@ -22,19 +22,7 @@ namespace engram {
 namespace {
 
 __device__ __forceinline__ int64_t load_id(const HashParams& p, int64_t raw) {
-  int64_t x = raw;
-  if (p.lookup != nullptr) {
-    if (raw < 0 || raw >= p.raw_vocab) {
-      set_status(p.status, ENGRAM_STATUS_ID_RANGE);
-      return p.pad_id;
-    }
-    x = __ldg(p.lookup + raw);
-  }
-  if (x < 0 || x >= p.vocab) {
-    set_status(p.status, ENGRAM_STATUS_ID_RANGE);
-    return p.pad_id;
-  }
-  return x;
+  return checked_id(raw, p.lookup, p.raw_vocab, p.vocab, p.pad_id, p.status);
 }
 
 __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashParams p) {
@@ -97,29 +85,6 @@ __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashP
   }
 }
 
-// Decode / chunked prefill: after the hash of this chunk has read the old ring,
-// the ring becomes the last n_hist ids of (old ring ++ chunk).  One thread per
-// sequence; it runs after hash_kernel on the same stream.
-__global__ void id_ring_kernel(const __grid_constant__ HashParams p) {
-  pdl_wait();  // the previous kernel on the stream has finished (PDL)
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= p.B) return;
-  if (p.id_ring_out != nullptr) {
-    int64_t* ring = p.id_ring_out + static_cast<int64_t>(b) * p.n_hist;
-    const int64_t base = static_cast<int64_t>(b) * p.T;
-    // ascending j reads index j + T >= j before writing j (in-place forward shift)
-    for (int j = 0; j < p.n_hist; ++j) {
-      int src = j + p.T;  // position in (old ring ++ chunk)
-      int64_t v;
-      if (src < p.n_hist) v = ring[src];
-      else v = load_id(p, __ldg(p.ids + base + (src - p.n_hist)));
-      ring[j] = v;
-    }
-  }
-  // the sequence has consumed this chunk; later kernels of the call read pos - T
-  if (p.pos_advance != nullptr) p.pos_advance[b] += p.T;
-}
-
 // Id at position t of sequence b (pad / history before the start), compressed
 // and range-checked.
 __device__ __forceinline__ uint64_t token_at(const HashParams& p, int b, int t) {
@@ -137,11 +102,12 @@ __device__ __forceinline__ uint64_t token_at(const HashParams& p, int b, int t) 
 
 // Absolute table row of row q = m*nh + h of e: the window of token m's order
 // (read through L1), xor of the products, Barrett reduction by head h's prime.
-__device__ __forceinline__ int64_t hashed_row(const HashParams& p, int q) {
-  const int m = q / p.nh;
+__device__ __forceinline__ int64_t hashed_row(const HashGatherParams& g, int q) {
+  const HashParams& p = g.h;
+  const int m = static_cast<int>(fast_div(static_cast<uint32_t>(q), g.div_nh));
   const int h = q - m * p.nh;
-  const int o = h / p.J;
-  const int b = m / p.T;
+  const int o = static_cast<int>(fast_div(static_cast<uint32_t>(h), g.div_J));
+  const int b = static_cast<int>(fast_div(static_cast<uint32_t>(m), g.div_T));
   const int t = m - b * p.T;
   const int n = p.orders[o];
   uint64_t mix = token_at(p, b, t) * p.mult[0];
@@ -167,7 +133,7 @@ __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant_
   const int q0 = ((static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x)) >> 5) * ROWS;
   if (q0 >= total) return;
   const int q = q0 + (lane % ROWS);
-  const int64_t row = q < total ? hashed_row(p, q) : 0;
+  const int64_t row = q < total ? hashed_row(g, q) : 0;
   const char* tab = static_cast<const char*>(g.table);
   if (CH > 0) {
     // piece i of the warp's rows is row i / CH, 16-byte column i % CH
@@ -236,15 +202,15 @@ cudaError_t launch_hash(const HashParams& p, cudaStream_t s) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (((p.id_ring_out != nullptr && p.n_hist > 0) || p.pos_advance != nullptr) && p.B > 0) {
-    launch_k(id_ring_kernel, dim3((p.B + 127) / 128), dim3(128), 0, s, p);
-    return cudaGetLastError();
-  }
   return cudaSuccess;
 }
 
-cudaError_t launch_hash_gather(const HashGatherParams& g, cudaStream_t s) {
+cudaError_t launch_hash_gather(const HashGatherParams& g0, cudaStream_t s) {
+  HashGatherParams g = g0;
   const HashParams& p = g.h;
+  g.div_nh = make_fastdiv(static_cast<uint32_t>(p.nh > 0 ? p.nh : 1));
+  g.div_J = make_fastdiv(static_cast<uint32_t>(p.J > 0 ? p.J : 1));
+  g.div_T = make_fastdiv(static_cast<uint32_t>(p.T > 0 ? p.T : 1));
   const int64_t total = static_cast<int64_t>(p.B) * p.T * p.nh;
   if (total > 0) {
     constexpr int kRows = 16;                    // rows per warp for 128-byte rows
@@ -258,10 +224,6 @@ cudaError_t launch_hash_gather(const HashGatherParams& g, cudaStream_t s) {
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-  }
-  if (((p.id_ring_out != nullptr && p.n_hist > 0) || p.pos_advance != nullptr) && p.B > 0) {
-    launch_k(id_ring_kernel, dim3((p.B + 127) / 128), dim3(128), 0, s, p);
-    return cudaGetLastError();
   }
   return cudaSuccess;
 }
