@@ -203,6 +203,20 @@ def algorithmic(w):
     }
 
 
+def max_over_ranks(t, world):
+    """Element-wise max over ranks of a float64 tensor of per-rank timings
+    (on the device of the process group's backend); identity for one rank."""
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t
+
+
+def job_throughput(world, units_per_step_per_rank, steps, max_ms):
+    """Whole-job units/s: every rank processes its own replica's units, timed
+    by the slowest rank."""
+    return world * units_per_step_per_rank * steps / (max_ms / 1e3)
+
+
 def run_ours(args, rank, world, device):
     from hashed_gram_conditional_hash_b200 import EngramLayer
     from hashed_gram_conditional_hash_b200 import _lib as L
@@ -297,12 +311,10 @@ def run_ours(args, rank, world, device):
     t_gate = sum(e["before_gate"].elapsed_time(e["before_conv"]) for e in ev)
     t_conv = sum(e["before_conv"].elapsed_time(e["after_conv"]) for e in ev)
     times = torch.tensor([t_step, t_proj, t_hash, t_gate, t_conv], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    t_step, t_proj, t_hash, t_gate, t_conv = times.tolist()
+    t_step, t_proj, t_hash, t_gate, t_conv = max_over_ranks(times, world).tolist()
 
     tokens_step = Bq * Tq
-    value = world * tokens_step * K / (t_step / 1e3)
+    value = job_throughput(world, tokens_step, K, t_step)
     a = algorithmic(w)
     proj_s = t_proj / K / 1e3
     proj_tflops = a["proj_flops"] * tokens_step / proj_s / 1e12
@@ -386,12 +398,10 @@ def run_e2e(args, layer, p, w, device, world):
     e1.record()
     torch.cuda.synchronize()
     t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms = t.item()
+    ms = max_over_ranks(t, world).item()
     h2d = ids_h.numel() * 8 + hid_h.numel() * hid_h.element_size()
     d2h = y_h.numel() * y_h.element_size()
-    return {"value": world * Bq * Tq * K / (ms / 1e3), "unit": "tokens/s",
+    return {"value": job_throughput(world, Bq * Tq, K, ms), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
