@@ -68,6 +68,8 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kEpiCols = kBN / 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_bf16(2 * kBM, kBN);
+constexpr uint32_t kIdescHalf = idesc_bf16(2 * kBM, kBN / 2);   // half-width V tiles (N = 128)
+constexpr int kBTileHalf = kBTile / 2;      // 8 KB: one K-block of a half tile's B (64 rows)
 constexpr int kMaxStages = 6;
 constexpr int kEpiRows = 32;                // token rows per epilogue warp
 constexpr int kXCols = 64;                  // columns per staged tile (128 bytes of bf16)
@@ -78,16 +80,70 @@ constexpr int kNumBars = 2 * kMaxStages + 2 + 2 + 2 + kEpiWarps;
 struct Tc2Params {
   ProjParams p;
   int32_t num_n_tiles, nv_tiles;
+  // tile order: M-block-major, an M-block's key tiles before its value tiles;
+  // the last n_split value tiles (all in M-blocks >= mb0, from value tile vb0
+  // of M-block mb0 on) run at the end as 2 * n_split half-width tiles, so that
+  // the last round of pairs is not left mostly idle
+  int32_t nk_tiles, n_split, mb0, vb0;
   int64_t num_tiles;                         // pair tiles
   uint64_t timeout_ns;
   int32_t force_timeout;
 };
 
+// One pair tile: its M-block, whether it is a key or value tile, and the
+// output / weight columns it covers.
+struct Tile {
+  int64_t mb;
+  bool is_v, half;
+  int kt;       // key tiles: index in [0, hc * H / 256) (branch kt / nv_tiles)
+  int col0;     // first output column of the tile: in H (value) or in hc*H (key)
+  int width;    // 256, or 128 for a half-width value tile
+};
+__device__ __forceinline__ Tile tile_at(const Tc2Params& tp, int64_t t) {
+  Tile x;
+  const int nk = tp.nk_tiles, nv = tp.nv_tiles, nn = tp.num_n_tiles;
+  const int64_t full_before = static_cast<int64_t>(tp.mb0) * nn;  // tiles of the M-blocks before mb0
+  const int64_t n_full = tp.num_tiles - 2 * static_cast<int64_t>(tp.n_split);
+  x.half = false;
+  x.width = kBN;
+  int r;                                   // index inside the M-block (keys, then values)
+  if (t >= n_full) {                       // half-width value tiles
+    const int64_t i = t - n_full;
+    const int64_t vidx = static_cast<int64_t>(tp.mb0) * nv + tp.vb0 + (i >> 1);
+    x.mb = vidx / nv;
+    x.is_v = true;
+    x.half = true;
+    x.width = kBN / 2;
+    x.kt = 0;
+    x.col0 = static_cast<int>(vidx - x.mb * nv) * kBN + static_cast<int>(i & 1) * (kBN / 2);
+    return x;
+  }
+  if (t < full_before) {
+    x.mb = t / nn;
+    r = static_cast<int>(t - x.mb * nn);
+  } else {
+    const int64_t u = t - full_before;
+    if (u < nk + tp.vb0) {
+      x.mb = tp.mb0;
+      r = static_cast<int>(u);
+    } else {                               // M-blocks after mb0 keep only their key tiles
+      const int64_t w = u - (nk + tp.vb0);
+      x.mb = tp.mb0 + 1 + w / nk;
+      r = static_cast<int>(w % nk);
+    }
+  }
+  x.is_v = r >= nk;
+  x.kt = x.is_v ? 0 : r;
+  x.col0 = (x.is_v ? r - nk : r) * kBN;
+  return x;
+}
+
 template <int KC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CUtensorMap map_a,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_k,
-                const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_vo) {
+                const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_vo,
+                const __grid_constant__ CUtensorMap map_vh) {
   constexpr int kABytes = KC * kATile;
   constexpr int kBBytes = KC * kBTile;
   constexpr int kStageBytes = kABytes + kBBytes;
@@ -164,6 +220,7 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_k)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_q)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_vo)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_vh)) : "memory");
     }
     uint64_t pol_w, pol_a;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_w));
@@ -173,10 +230,12 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
     uint32_t pending = 0, pend_par = 0;      // stages armed by the leader (drain on abort)
     bool ok = true;
     for (int64_t tile = pair; tile < tp.num_tiles && ok; tile += npairs) {
-      const int64_t m0 = (tile / tp.num_n_tiles) * (2 * kBM) + rank * kBM;
-      const int nb = static_cast<int>(tile % tp.num_n_tiles);
-      const bool is_v = nb < tp.nv_tiles;
-      const int32_t yb = (is_v ? nb : nb - tp.nv_tiles) * kBN + static_cast<int32_t>(rank) * kBNh;
+      const Tile tl = tile_at(tp, tile);
+      const int64_t m0 = tl.mb * (2 * kBM) + rank * kBM;
+      // this CTA's weight rows: half of the tile's output columns
+      const int32_t yb = tl.col0 + static_cast<int32_t>(rank) * (tl.width / 2);
+      const CUtensorMap* bmap = tl.half ? &map_vh : (tl.is_v ? &map_v : &map_k);
+      const uint32_t tx = 2u * (kABytes + (tl.half ? KC * kBTileHalf : kBBytes));   // both CTAs' bytes
       for (int kb = 0; kb < p.nh; kb += KC) {
         ok = wait_pair(empty_bar(stage), phase ^ 1u);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -184,16 +243,16 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
           const uint32_t sa = base + stage * kStageBytes;
           const uint32_t lbar = mapa_shared(full_bar(stage), 0);
           if (leader) {
-            mbar_arrive_expect_tx(full_bar(stage), 2 * kStageBytes);
+            mbar_arrive_expect_tx(full_bar(stage), tx);
             pending |= 1u << stage;
             pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
           }
           if (KC == 1) {
             tma_load_2d_pair(sa, &map_a, kb * kBK, static_cast<int32_t>(m0), lbar, pol_a);
-            tma_load_2d_pair(sa + kABytes, is_v ? &map_v : &map_k, kb * kBK, yb, lbar, pol_w);
+            tma_load_2d_pair(sa + kABytes, bmap, kb * kBK, yb, lbar, pol_w);
           } else {
             tma_load_3d_pair(sa, &map_a, 0, static_cast<int32_t>(m0), kb, lbar, pol_a);
-            tma_load_3d_pair(sa + kABytes, is_v ? &map_v : &map_k, 0, yb, kb, lbar, pol_w);
+            tma_load_3d_pair(sa + kABytes, bmap, 0, yb, kb, lbar, pol_w);
           }
         }
         __syncwarp();
@@ -222,6 +281,9 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
         if (!ok) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        const bool half = tile_at(tp, tile).half;
+        const uint32_t idesc = half ? kIdescHalf : kIdesc;
+        const int btile = half ? kBTileHalf : kBTile;
         for (int kb = 0; kb < p.nh; kb += KC) {
           ok = wait_pair(full_bar(stage), phase);
           if (!ok) break;
@@ -233,7 +295,7 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
 #pragma unroll
             for (int k = 0; k < kBK / 16; ++k)
               tc_mma_pair(d_tmem, umma_desc_sw128(sa + j * kATile + k * 32),
-                          umma_desc_sw128(sb + j * kBTile + k * 32), kIdesc,
+                          umma_desc_sw128(sb + j * btile + k * 32), idesc,
                           (kb > 0 || j > 0 || k > 0) ? 1u : 0u);
           tc_commit_pair(empty_bar(stage), 0x3);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -271,15 +333,15 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
       q_inflight = true;
     };
     for (int64_t tile = pair; tile < tp.num_tiles; tile += npairs) {
-      const int64_t tok0 = (tile / tp.num_n_tiles) * (2 * kBM) + rank * kBM + quad * kEpiRows;
+      const Tile tl = tile_at(tp, tile);
+      const int64_t tok0 = tl.mb * (2 * kBM) + rank * kBM + quad * kEpiRows;
       const int64_t m = tok0 + lane;
-      const int nb = static_cast<int>(tile % tp.num_n_tiles);
       const bool live = m < p.M;
-      const bool is_v = nb < tp.nv_tiles;
-      const int kt = nb - tp.nv_tiles;
-      const int h = is_v ? 0 : kt / tp.nv_tiles;
-      const int c0 = is_v ? nb * kBN : (kt - h * tp.nv_tiles) * kBN;  // first column in H
-      const int cc = c0 + half * kEpiCols;                               // this warp's first
+      const bool is_v = tl.is_v;
+      const int h = is_v ? 0 : tl.kt / tp.nv_tiles;
+      const int c0 = is_v ? tl.col0 : tl.col0 - h * p.H;                // first column in H
+      const int wcols = tl.width / 2;                                    // columns per warp
+      const int cc = c0 + half * wcols;                                  // this warp's first
       if (!is_v) {
         fill_q(cc, h, static_cast<int32_t>(tok0));
         if (lane == 0) tma_prefetch_l2_3d(&map_q, cc + kXCols, h, static_cast<int32_t>(tok0));
@@ -288,12 +350,12 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                             static_cast<uint32_t>(acc * kBN + half * kEpiCols);
+                             static_cast<uint32_t>(acc * kBN + half * wcols);
       bool fine = true;
       if (is_v && tok0 < p.M) {  // (a warp whose rows all lie past M stores nothing)
         // V -> bf16 into the staging tile (swizzled rows), then one tensor store per 64 columns
 #pragma unroll 1
-        for (int f = 0; f < kEpiCols / kXCols; ++f) {
+        for (int f = 0; f < wcols / kXCols; ++f) {
           if (lane == 0) bulk_wait_group_read0();  // the previous store has left the tile
           __syncwarp();
 #pragma unroll
@@ -471,6 +533,39 @@ bool make_map_hidden(CUtensorMap* map, const void* base, uint64_t H, uint64_t hc
 template <int KC>
 cudaError_t launch_kc(const Tc2Params& tp, const ProjParams& p, cudaStream_t s);
 
+// CTA pairs of proj_tc2_kernel<KC> resident at once on the current device
+// (cached per device; also sets the kernel's shared-memory attribute).
+template <int KC>
+int resident_pairs_kc() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  if (cudaFuncSetAttribute(proj_tc2_kernel<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSmemBytes)) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, proj_tc2_kernel<KC>, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();  // clear; fall back to one pair per two SMs
+    n = num_sms() / 2;
+  }
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
 }  // namespace
 
 // Dense A (rows == null), bf16, Dh == 64, H % 256 == 0; grid of CTA pairs.
@@ -482,9 +577,19 @@ cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s) {
   Tc2Params tp;
   tp.p = p;
   tp.nv_tiles = p.H / kBN;
+  tp.nk_tiles = p.hc * tp.nv_tiles;
   tp.num_n_tiles = (1 + p.hc) * tp.nv_tiles;
   const int64_t m2 = (p.M + 2 * kBM - 1) / (2 * kBM);
-  tp.num_tiles = m2 * tp.num_n_tiles;
+  const int64_t full = m2 * tp.num_n_tiles;
+  // split the tail of value tiles when the last round of pairs would run
+  // at most half full (the pair count is known once the grid is sized)
+  const int64_t pairs = (p.nh % 2 == 0) ? resident_pairs_kc<2>() : resident_pairs_kc<1>();
+  const int64_t rem = pairs > 0 ? full % pairs : 0;
+  tp.n_split = (rem > 0 && 2 * rem <= pairs && rem <= m2 * tp.nv_tiles) ? static_cast<int32_t>(rem) : 0;
+  const int64_t first_split = m2 * tp.nv_tiles - tp.n_split;   // value-tile index of the first split tile
+  tp.mb0 = static_cast<int32_t>(first_split / tp.nv_tiles);
+  tp.vb0 = static_cast<int32_t>(first_split % tp.nv_tiles);
+  tp.num_tiles = full + tp.n_split;                                // n_split full tiles become 2 * n_split
   tp.force_timeout = (p.debug & ENGRAM_DEBUG_FORCE_TIMEOUT) ? 1 : 0;
   tp.timeout_ns = tp.force_timeout ? 20000000ull : 2000000000ull;
   // two K-blocks per TMA box when the head count allows it
@@ -511,41 +616,18 @@ cudaError_t launch_kc(const Tc2Params& tp, const ProjParams& p, cudaStream_t s) 
   ok = ok && make_map_hidden(&map_q, p.hidden, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.hc),
                              static_cast<uint64_t>(p.M)) &&
        make_map2(&map_vo, p.V, static_cast<uint64_t>(p.H), static_cast<uint64_t>(p.M), kXCols, kEpiRows);
+  // half-width value tiles: 64 weight rows per CTA
+  CUtensorMap map_vh;
+  ok = ok && (KC == 1 ? make_map2(&map_vh, p.w_value, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.H), kBK,
+                                  kBNh / 2)
+                      : make_map3(&map_vh, p.w_value, static_cast<uint64_t>(p.E), static_cast<uint64_t>(p.H),
+                                  kBNh / 2, KC));
   if (!ok) return cudaErrorInvalidValue;
-  static bool attr_set[64] = {false};
-  static int max_pairs[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(proj_tc2_kernel<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
-  // as many pairs as can be resident at once (not every SM pair need form a cluster)
-  if (dev >= 0 && dev < 64 && max_pairs[dev] == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(num_sms() & ~1), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, proj_tc2_kernel<KC>, &cfg) != cudaSuccess || n <= 0) {
-      cudaGetLastError();  // clear; fall back to one pair per two SMs
-      n = num_sms() / 2;
-    }
-    max_pairs[dev] = n;
-  }
-  int64_t pairs = (dev >= 0 && dev < 64) ? max_pairs[dev] : num_sms() / 2;
+  int64_t pairs = resident_pairs_kc<KC>();
+  if (pairs <= 0) return cudaErrorInvalidValue;
   if (pairs > tp.num_tiles) pairs = tp.num_tiles;
   launch_k(proj_tc2_kernel<KC>, dim3(static_cast<unsigned>(2 * pairs)), dim3(kThreads), kSmemBytes, s, tp, map_a, map_v, map_k,
-           map_q, map_vo);
+           map_q, map_vo, map_vh);
   return cudaGetLastError();
 }
 

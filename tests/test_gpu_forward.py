@@ -94,6 +94,19 @@ def test_forward_zero_conv_is_gated_value():
     assert rel_err(y.double().cpu().numpy(), ref["g"][..., None] * ref["V"][:, :, None, :]) <= TOL["bf16"]
 
 
+def test_forward_split_value_tail_tiles():
+    # 2 M-blocks x 40 column tiles = 80 pair tiles: the 6 left for a last
+    # round of pairs run as 12 half-width value tiles
+    w = W.small_workload(B=2, T=256, hidden=2048, hc_mult=4)
+    p = device_params(w)
+    y = _run(p, "auto")
+    ref = oracle_forward_full(p)
+    assert rel_err(y.double().cpu().numpy(), ref["Y"]) <= TOL[w.dtype]
+    # the same rows through the single-CTA engine (no tile split)
+    d = _run(p, "single_cta").double()
+    assert (y.double() - d).abs().max().item() <= 1e-2 * d.abs().max().item()
+
+
 def test_forward_engines_agree():
     w = W.small_workload(B=2, T=300, hidden=512, hc_mult=4)
     p = device_params(w)
