@@ -135,6 +135,7 @@ int64_t rows_ld(int64_t M) { return (M + 127) / 128 * 128; }
 struct ForwardLayout {
   size_t e_off, rows_off;
   StageLayout st;
+  size_t wp_off, end;       // norm_key * norm_query [hc, H] float, then the end
 };
 ForwardLayout forward_layout(const engram_config* c, int64_t M) {
   ForwardLayout L;
@@ -145,6 +146,8 @@ ForwardLayout forward_layout(const engram_config* c, int64_t M) {
   const size_t e_end = align256(static_cast<size_t>(M) * nh * c->row_dim * es);
   const size_t rows_end = align256(static_cast<size_t>(nh) * rows_ld(M) * sizeof(int32_t));
   L.st = stage_layout(c, M, e_end > rows_end ? e_end : rows_end);
+  L.wp_off = L.st.end;
+  L.end = align256(L.wp_off + static_cast<size_t>(c->hc_mult) * c->hidden * sizeof(float));
   return L;
 }
 
@@ -430,7 +433,7 @@ engram_status engram_forward_workspace_size(const engram_config* cfg, int32_t B,
   engram_status st = check_config(cfg);
   if (st != ENGRAM_OK) return st;
   if (B < 0 || T < 0 || bytes == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "bad B/T/bytes");
-  *bytes = forward_layout(cfg, static_cast<int64_t>(B) * T).st.end;
+  *bytes = forward_layout(cfg, static_cast<int64_t>(B) * T).end;
   return ENGRAM_OK;
 }
 
@@ -492,8 +495,8 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
     if (!aligned16(state->v_ring)) return fail(ENGRAM_ERR_INVALID_ARG, "state v_ring must be 16-byte aligned");
   }
   const ForwardLayout L = forward_layout(cfg, M);
-  if (ws_bytes < L.st.end)
-    return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", ws_bytes, L.st.end);
+  if (ws_bytes < L.end)
+    return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", ws_bytes, L.end);
   char* w = static_cast<char*>(ws);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -524,6 +527,11 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
     hg.table = wts->table;
     hg.e = e;
     hg.row_bytes = row_bytes;
+    // the score's RMSNorm weight products, once per call, for the projection
+    hg.nk = static_cast<const uint16_t*>(wts->norm_key);
+    hg.nq = static_cast<const uint16_t*>(wts->norm_query);
+    hg.wprod = cfg->dtype == ENGRAM_BF16 ? reinterpret_cast<float*>(w + L.wp_off) : nullptr;
+    hg.n_w = cfg->hc_mult * cfg->hidden;
     st = cuda_check(launch_hash_gather(hg, s), "hash+gather");
   }
   if (st != ENGRAM_OK) return st;
@@ -542,6 +550,7 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   pp.hidden = hidden;
   pp.V = w + L.st.v_off;
   pp.partials = reinterpret_cast<float4*>(w + L.st.part_off);
+  pp.wprod = (!fused && cfg->dtype == ENGRAM_BF16) ? reinterpret_cast<const float*>(w + L.wp_off) : nullptr;
   pp.status = dev_status;
   pp.M = M;
   pp.nh = hp.nh;

@@ -67,6 +67,11 @@ struct HashGatherParams {
   void* e;                  // [B*T, nh*Dh]
   int32_t row_bytes;
   FastDiv div_nh, div_J, div_T;   // set by launch_hash_gather
+  // optional side job for the projection that follows: wprod[i] = nk[i] * nq[i]
+  const uint16_t* nk;
+  const uint16_t* nq;
+  float* wprod;             // [n_w] or null
+  int32_t n_w;
 };
 cudaError_t launch_hash_gather(const HashGatherParams& p, cudaStream_t s);
 
@@ -101,6 +106,7 @@ struct ProjParams {
   const void* hidden;       // [M, hc, H]
   void* V;                  // [M, H]
   float4* partials;         // [M, hc, n_tiles]
+  const float* wprod;       // [hc, H] norm_key * norm_query, or null (formed on the fly)
   uint32_t* status;
   int64_t M;
   int32_t nh, Dh, E, H, hc;

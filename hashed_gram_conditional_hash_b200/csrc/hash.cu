@@ -128,9 +128,13 @@ __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant_
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const HashParams& p = g.h;
   const int lane = threadIdx.x & 31;
+  const int gtid = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+  if (g.wprod != nullptr)   // the RMSNorm weight products of the score, for the projection
+    for (int i = gtid; i < g.n_w; i += static_cast<int>(gridDim.x * blockDim.x))
+      g.wprod[i] = bf16_to_f32(__ldg(g.nk + i)) * bf16_to_f32(__ldg(g.nq + i));
   // rows of e (B*T*nh) stay below 2^31 (checked by the launcher): 32-bit math
   const int total = p.B * p.T * p.nh;
-  const int q0 = ((static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x)) >> 5) * ROWS;
+  const int q0 = (gtid >> 5) * ROWS;
   if (q0 >= total) return;
   const int q = q0 + (lane % ROWS);
   const int64_t row = q < total ? hashed_row(g, q) : 0;

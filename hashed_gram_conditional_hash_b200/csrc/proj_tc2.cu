@@ -376,7 +376,9 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
           }
         }
       } else if (!is_v) {
-        float dot = 0.f, ssk = 0.f, ssq = 0.f;
+        // two columns per instruction: even and odd columns accumulate in the
+        // two lanes of each pair and are added at the end
+        float2 dot2 = make_float2(0.f, 0.f), ssk2 = dot2, ssq2 = dot2;
 #pragma unroll 1
         for (int f = 0; f < kEpiCols / kXCols && fine; ++f) {
           if (f > 0) {
@@ -392,31 +394,41 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
             const int col = cc + f * kXCols + c2 * 32;
             float k[32];
             tmem_ld32(taddr + (f * kXCols + c2 * 32), k);
-            const uint4* nk4 = reinterpret_cast<const uint4*>(nk + static_cast<int64_t>(h) * p.H + col);
-            const uint4* nq4 = reinterpret_cast<const uint4*>(nq + static_cast<int64_t>(h) * p.H + col);
+            const int64_t wi = static_cast<int64_t>(h) * p.H + col;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const uint4 qq = ld_shared_v4(xb + sw128_offset(lane, c2 * 4 + q));
-              const uint4 ka = __ldg(nk4 + q), qa = __ldg(nq4 + q);
+              float w[8];                       // nk * nq of the 8 columns
+              if (p.wprod != nullptr) {
+                const float4 wa = __ldg(reinterpret_cast<const float4*>(p.wprod + wi) + 2 * q);
+                const float4 wb = __ldg(reinterpret_cast<const float4*>(p.wprod + wi) + 2 * q + 1);
+                w[0] = wa.x; w[1] = wa.y; w[2] = wa.z; w[3] = wa.w;
+                w[4] = wb.x; w[5] = wb.y; w[6] = wb.z; w[7] = wb.w;
+              } else {
+                const uint4 ka = __ldg(reinterpret_cast<const uint4*>(nk + wi) + q);
+                const uint4 qa = __ldg(reinterpret_cast<const uint4*>(nq + wi) + q);
+                const uint32_t kw[4] = {ka.x, ka.y, ka.z, ka.w};
+                const uint32_t nw[4] = {qa.x, qa.y, qa.z, qa.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  w[2 * i] = __uint_as_float(kw[i] << 16) * __uint_as_float(nw[i] << 16);
+                  w[2 * i + 1] = __uint_as_float(kw[i] & 0xffff0000u) * __uint_as_float(nw[i] & 0xffff0000u);
+                }
+              }
               const uint32_t qw[4] = {qq.x, qq.y, qq.z, qq.w};
-              const uint32_t kw[4] = {ka.x, ka.y, ka.z, ka.w};
-              const uint32_t nw[4] = {qa.x, qa.y, qa.z, qa.w};
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                const float q0 = __uint_as_float(qw[i] << 16), q1 = __uint_as_float(qw[i] & 0xffff0000u);
-                const float w0 = __uint_as_float(kw[i] << 16) * __uint_as_float(nw[i] << 16);
-                const float w1 = __uint_as_float(kw[i] & 0xffff0000u) * __uint_as_float(nw[i] & 0xffff0000u);
-                const float k0 = k[8 * q + 2 * i], k1 = k[8 * q + 2 * i + 1];
-                dot = fmaf(k0 * w0, q0, dot);
-                dot = fmaf(k1 * w1, q1, dot);
-                ssk = fmaf(k0, k0, ssk);
-                ssk = fmaf(k1, k1, ssk);
-                ssq = fmaf(q0, q0, ssq);
-                ssq = fmaf(q1, q1, ssq);
+                const float2 q2 = make_float2(__uint_as_float(qw[i] << 16), __uint_as_float(qw[i] & 0xffff0000u));
+                const float2 k2 = make_float2(k[8 * q + 2 * i], k[8 * q + 2 * i + 1]);
+                const float2 kw2 = __fmul2_rn(k2, make_float2(w[2 * i], w[2 * i + 1]));
+                dot2 = __ffma2_rn(kw2, q2, dot2);
+                ssk2 = __ffma2_rn(k2, k2, ssk2);
+                ssq2 = __ffma2_rn(q2, q2, ssq2);
               }
             }
           }
         }
+        const float dot = dot2.x + dot2.y, ssk = ssk2.x + ssk2.y, ssq = ssq2.x + ssq2.y;
         if (fine && live)
           p.partials[(m * p.hc + h) * p.n_tiles + cc / kEpiCols] = make_float4(dot, ssk, ssq, 0.f);
       }
