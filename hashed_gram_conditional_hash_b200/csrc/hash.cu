@@ -117,6 +117,15 @@ __device__ __forceinline__ int64_t hashed_row(const HashGatherParams& g, int q) 
   return p.row_off[h] + static_cast<int64_t>(barrett_mod(mix, p.prime[h], p.barrett[h]));
 }
 
+// A 16-byte piece of a table row: read once, so it bypasses L1.
+__device__ __forceinline__ int4 ld_row_piece(const int4* p) {
+  int4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.s32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 // One warp produces ROWS (16 or 32) consecutive rows of e (row q = m*nh + h):
 // lane l < ROWS hashes row l, then the warp copies the table rows with every
 // 16-byte load issued before the stores.  CH = 16-byte pieces per row when
@@ -148,7 +157,7 @@ __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant_
       const int i = u * 32 + lane;
       const int r = i / CH;
       const int64_t src = __shfl_sync(0xffffffffu, row, r);
-      if (q0 + r < total) v[u] = __ldg(reinterpret_cast<const int4*>(tab + src * (CH * 16)) + (i - r * CH));
+      if (q0 + r < total) v[u] = ld_row_piece(reinterpret_cast<const int4*>(tab + src * (CH * 16)) + (i - r * CH));
     }
     int4* out = static_cast<int4*>(g.e) + static_cast<int64_t>(q0) * CH;
 #pragma unroll

@@ -358,16 +358,13 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
         for (int f = 0; f < wcols / kXCols; ++f) {
           if (lane == 0) bulk_wait_group_read0();  // the previous store has left the tile
           __syncwarp();
+          float v[kXCols];
+          tmem_ld64(taddr + f * kXCols, v);
 #pragma unroll
-          for (int c2 = 0; c2 < kXCols / 32; ++c2) {
-            float v[32];
-            tmem_ld32(taddr + (f * kXCols + c2 * 32), v);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              st_shared_v4(xb + sw128_offset(lane, c2 * 4 + q),
-                           make_uint4(bf16x2(v[8 * q + 0], v[8 * q + 1]), bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                      bf16x2(v[8 * q + 4], v[8 * q + 5]), bf16x2(v[8 * q + 6], v[8 * q + 7])));
-          }
+          for (int q = 0; q < kXCols / 8; ++q)
+            st_shared_v4(xb + sw128_offset(lane, q),
+                         make_uint4(bf16x2(v[8 * q + 0], v[8 * q + 1]), bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                    bf16x2(v[8 * q + 4], v[8 * q + 5]), bf16x2(v[8 * q + 6], v[8 * q + 7])));
           fence_proxy_async();  // the tile's generic writes are visible to the tensor store
           __syncwarp();
           if (lane == 0) {
@@ -389,11 +386,12 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
           if (!fine) break;
           q_inflight = false;
           q_par ^= 1u;
+          float kf[kXCols];
+          tmem_ld64(taddr + f * kXCols, kf);
 #pragma unroll
           for (int c2 = 0; c2 < kXCols / 32; ++c2) {
             const int col = cc + f * kXCols + c2 * 32;
-            float k[32];
-            tmem_ld32(taddr + (f * kXCols + c2 * 32), k);
+            const float* k = kf + c2 * 32;
             const int64_t wi = static_cast<int64_t>(h) * p.H + col;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {

@@ -73,3 +73,23 @@ def test_chunked_prefill_with_state(chunks):
     err = (y.double() - y_full.double()).abs().max().item()
     assert err <= 1e-2 * y_full.double().abs().max().item()
     assert torch.all(state.pos == t0)
+
+
+def test_streaming_with_raw_ids_keeps_compressed_ids_in_the_ring():
+    # raw ids go through the lookup; the ring keeps the compressed ids the
+    # hash needs for the next chunk (decode steps, then one long chunk)
+    w = W.small_workload(B=3, T=80, raw_vocab=6500, orders=(2, 3, 4), dilation=4, hidden=256, hc_mult=2)
+    p = device_params(w)
+    layer = EngramLayer.from_params(p)
+    y_full = layer.forward(p.ids, p.hidden)
+    state = layer.new_state(w.B)
+    outs, t0 = [], 0
+    for n in (1,) * 5 + (75,):
+        outs.append(layer.forward(p.ids[:, t0:t0 + n].contiguous(), p.hidden[:, t0:t0 + n].contiguous(),
+                                  state=state))
+        t0 += n
+    y = torch.cat(outs, 1)
+    err = (y.double() - y_full.double()).abs().max().item()
+    assert err <= 1e-2 * y_full.double().abs().max().item()
+    assert torch.equal(state.id_ring, p.lookup[p.ids[:, -(w.max_n - 1):]])
+    assert torch.all(state.pos == w.T)

@@ -47,6 +47,7 @@ SMALL = [
     dict(B=1, T=150, dilation=9, hc_mult=3),                      # long halo (R = 27)
     dict(B=2, T=45, row_dim=20),                                  # 40-byte rows
     dict(B=2, T=90, hc_mult=6, hidden=128),                       # more than 4 branches
+    dict(B=2, T=60, raw_vocab=6500),                              # raw ids through the lookup
     dict(B=2, T=41, row_dim=32),                                  # 64-byte rows (generic gather)
     dict(B=1, T=37, row_dim=128, orders=(2, 3, 4)),               # 256-byte rows (generic gather)
 ]
