@@ -45,6 +45,12 @@
 // for KC = 2; 6 stages of 32 KB for KC = 1, used when the head count is odd).
 // Every wait is bounded; an abort raises the flag in both CTAs; no multicast
 // loads are used anywhere (only the commit arrives on both CTAs' barriers).
+//
+// Tiles run M-block-major (an M-block's key tiles, then its value tiles) over
+// a persistent grid of as many pairs as fit; when the last round of pairs
+// would be at most half full, that many value tiles from the end run as twice
+// as many 256 x 128 tiles (N = 128 MMA, 64 weight rows per CTA).  The key
+// epilogue takes norm_key * norm_query from a per-call fp32 table when given.
 #include <cuda.h>
 
 #include "engram_internal.cuh"

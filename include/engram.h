@@ -54,7 +54,7 @@ extern "C" {
 typedef enum {
   ENGRAM_OK = 0,
   ENGRAM_ERR_INVALID_ARG = 1, /* null pointer, bad size, range, alignment */
-  ENGRAM_ERR_UNSUPPORTED = 2, /* valid but not supported by this build (dtype/shape) */
+  ENGRAM_ERR_UNSUPPORTED = 2, /* valid, but a dtype or shape the library does not handle */
   ENGRAM_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
   ENGRAM_ERR_TIMEOUT = 4,     /* device reported ENGRAM_STATUS_TIMEOUT */
   ENGRAM_ERR_ID_RANGE = 5     /* device reported ENGRAM_STATUS_ID_RANGE / _ROW_RANGE */
