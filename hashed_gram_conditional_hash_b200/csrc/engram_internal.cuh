@@ -167,6 +167,7 @@ struct ConvParams {
   int32_t tile_t;           // positions per block of the tile form (set by launch_gated_conv)
   // thread decode of the run form (set by launch_gated_conv)
   FastDiv div_b, div_cls, div_run, div_cg;
+  FastDiv div_ring;         // ring_len, for the decode step (set by launch_gated_conv)
 };
 cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s);
 // True when launch_gated_conv also writes the chunk's V/g rows into the state

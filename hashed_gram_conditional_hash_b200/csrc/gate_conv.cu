@@ -548,44 +548,44 @@ __global__ void __launch_bounds__((kTileC / CPL) * ENGRAM_MAX_HC) conv_tile_kern
 
 // One decode step (T = 1) with the streaming state, K = 4 taps, bfloat16,
 // 256-channel slices: block (sequence b, slice), one warp per branch, 8
-// channels per lane.  Thread 0 turns pos into the ring rows of the taps at
-// t - 3 dil, t - 2 dil, t - dil (the ring holds (K-1) dil + 1 >= 3 dil + 1
-// positions, slot = position mod ring length); then every lane loads its
-// 16-byte pieces of V(t) and of those three ring rows, the four gates and its
-// taps, and stores 8 channels of Y.  The same kernel is the step's state
-// advance: the branch-0 warp writes V(t) and lanes 0 write g(t) into t's
-// slot, which no tap of this step reads.
+// channels per lane.  Every lane loads its 16-byte piece of V(t) and the
+// step's gate, turns pos into the ring rows of the taps at t - 3 dil,
+// t - 2 dil, t - dil itself (the ring holds (K-1) dil + 1 >= 3 dil + 1
+// positions, slot = position mod ring length, by invariant-divisor
+// multiplication), loads its pieces of those three rows, their gates and its
+// taps, and stores 8 channels of Y; no block barrier.  The same kernel is the
+// step's state advance: the branch-0 warp writes V(t) and lanes 0 write g(t)
+// into t's slot, which no tap of this step reads.
 __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __grid_constant__ ConvParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   constexpr int K = 4;
-  __shared__ int64_t s_row[K];   // ring row (b * ring_len + slot) of tap i; -1 before the start
   const int b = static_cast<int>(blockIdx.x);
   const int tid = static_cast<int>(threadIdx.x);
   const int h = tid >> 5, lane = tid & 31;
-  const bool worker = h < p.hc;
+  if (h >= p.hc) return;
   const int c = static_cast<int>(blockIdx.y) * kTileC + lane * 8;
   const uint16_t* V = static_cast<const uint16_t*>(p.V);
   uint16_t* vr = static_cast<uint16_t*>(const_cast<void*>(p.v_ring));
   float* gr = const_cast<float*>(p.g_ring);
-  if (tid == 0) {
-    const int64_t P = __ldg(p.pos + b) - p.pos_lag;   // position of this step's token
-    const int64_t slot_t = P % p.ring_len;
-#pragma unroll
-    for (int i = 0; i < K; ++i) {                     // tap i sits at t - (K-1-i) dil
-      const int64_t back = static_cast<int64_t>(K - 1 - i) * p.dil;
-      int64_t slot = slot_t - back;
-      if (slot < 0) slot += p.ring_len;
-      s_row[i] = (P - back >= 0) ? static_cast<int64_t>(b) * p.ring_len + slot : -1;
-    }
-  }
-  __syncthreads();
-  if (!worker) return;
   uint4 raw[K];
   float gg[K];
+  // what does not depend on the ring first, then every thread turns pos into
+  // the ring rows of its taps itself (no block barrier on the way)
+  raw[K - 1] = __ldg(reinterpret_cast<const uint4*>(V + static_cast<int64_t>(b) * p.H + c));
+  gg[K - 1] = __ldg(p.g + static_cast<int64_t>(b) * p.hc + h);
+  const int64_t P = __ldg(p.pos + b) - p.pos_lag;   // position of this step's token
+  const int64_t slot_t = (P >= 0 && P < INT32_MAX)
+                             ? static_cast<int64_t>(P - static_cast<int64_t>(fast_div(static_cast<uint32_t>(P), p.div_ring)) *
+                                                            p.ring_len)
+                             : P % p.ring_len;
+  const int64_t ring0 = static_cast<int64_t>(b) * p.ring_len;
 #pragma unroll
-  for (int i = 0; i < K - 1; ++i) {
-    const int64_t row = s_row[i];
-    if (row >= 0) {
+  for (int i = 0; i < K - 1; ++i) {                 // tap i sits at t - (K-1-i) dil
+    const int64_t back = static_cast<int64_t>(K - 1 - i) * p.dil;
+    int64_t slot = slot_t - back;
+    if (slot < 0) slot += p.ring_len;
+    if (P - back >= 0) {
+      const int64_t row = ring0 + slot;
       raw[i] = __ldg(reinterpret_cast<const uint4*>(vr + row * p.H + c));
       gg[i] = __ldg(gr + row * p.hc + h);
     } else {
@@ -593,8 +593,6 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __g
       gg[i] = 0.f;
     }
   }
-  raw[K - 1] = __ldg(reinterpret_cast<const uint4*>(V + static_cast<int64_t>(b) * p.H + c));
-  gg[K - 1] = __ldg(p.g + static_cast<int64_t>(b) * p.hc + h);
   float2 w2[4][K];                                // [channel pair][tap]
   {
     float w[8][K];
@@ -623,7 +621,7 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __g
   }
   Pair8<uint16_t>::store(static_cast<uint16_t*>(p.Y) + (static_cast<int64_t>(b) * p.hc + h) * p.H + c, acc);
   // the step's state advance
-  const int64_t row_t = s_row[K - 1];
+  const int64_t row_t = ring0 + slot_t;
   if (h == 0) *reinterpret_cast<uint4*>(vr + row_t * p.H + c) = raw[K - 1];
   if (blockIdx.y == 0 && lane == 0) gr[row_t * p.hc + h] = gg[K - 1];
 }
@@ -741,8 +739,10 @@ cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
   if (p.B <= 0 || p.T <= 0) return cudaSuccess;
   if (p.H % 8 != 0) return cudaErrorInvalidValue;
   if (conv_writes_rings(p)) {
+    ConvParams q = p;
+    q.div_ring = make_fastdiv(static_cast<uint32_t>(p.ring_len));
     launch_k(conv_step_kernel, dim3(static_cast<unsigned>(p.B), static_cast<unsigned>(p.H / kTileC)),
-             dim3(32 * p.hc), 0, s, p);
+             dim3(32 * p.hc), 0, s, q);
     return cudaGetLastError();
   }
   const int64_t threads = static_cast<int64_t>(p.B) * p.T * (p.H / 8);
