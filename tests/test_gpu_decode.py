@@ -41,7 +41,7 @@ def test_decode_workload_matches_oracle_and_prefill():
     ys, state = _decode_all(layer, p.ids, p.hidden)
     S, B = w.decode_calls, w.B
     # oracle: the prefill over the 256-token sequences at sampled positions
-    pos = sample_positions(B, S, w.dil, 24, seed=5)
+    pos = sample_positions(B, S, w.dil, 4096, seed=5)
     Yref, _, _, _ = oracle_at(p, pos, hidden_bt=lambda b, t: p.hidden[torch.from_numpy(t).to(DEV),
                                                                          torch.from_numpy(b).to(DEV)])
     got = torch.stack([ys[t, b] for b, t in pos]).double().cpu().numpy()

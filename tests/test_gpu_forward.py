@@ -10,8 +10,9 @@ from hashed_gram_conditional_hash_b200 import EngramLayer
 from hashed_gram_conditional_hash_b200 import _lib as L
 from hashed_gram_conditional_hash_b200 import workloads as W
 
-from gpu_helpers import (TOL, device_params, oracle_at, oracle_forward_full, rel_err,
+from gpu_helpers import (TOL, device_params, oracle_at, oracle_forward_full, oracle_ids, rel_err,
                          sample_positions)
+from oracle import engram_oracle as O
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -72,18 +73,40 @@ def test_forward_tiny_f32_full():
     assert err <= TOL["f32"], err
 
 
-@pytest.mark.parametrize("name,n_random", [("model_bf16", 48), ("large_table_bf16", 24),
-                                           ("hbm_table_bf16", 16)])
-@pytest.mark.parametrize("engine", ["auto", "single_cta"])
-def test_forward_full_size_sampled(name, n_random, engine):
+@pytest.mark.parametrize("name", ["model_bf16", "large_table_bf16", "hbm_table_bf16"])
+def test_forward_full_size_sampled(name):
+    # the bench's launch configuration at full size: both tensor-core engines
+    # against the oracle at the sequence edges plus 4096 random positions
     w = W.CONFIGS[name]
     p = device_params(w)
-    y = _run(p, engine)
-    pos = sample_positions(w.B, w.T, w.dil, n_random, seed=11)
-    Yref, s, g, _ = oracle_at(p, pos)
-    got = torch.stack([y[b, t] for b, t in pos]).double().cpu().numpy()
-    err = rel_err(got, Yref)
-    assert err <= TOL[w.dtype], err
+    pos = sample_positions(w.B, w.T, w.dil, 4096, seed=11)
+    Yref, _, _, _ = oracle_at(p, pos)
+    bi = torch.tensor([b for b, _ in pos], device=DEV)
+    ti = torch.tensor([t for _, t in pos], device=DEV)
+    for engine in ("auto", "single_cta"):
+        y = _run(p, engine)
+        err = rel_err(y[bi, ti].double().cpu().numpy(), Yref)
+        assert err <= TOL[w.dtype], (engine, err)
+        del y
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "model_bf16", "large_table_bf16", "hbm_table_bf16"])
+def test_gathered_rows_full_size_bit_exact(name):
+    # white-box: on the gather-then-project path the forward's workspace starts
+    # with e [M, E]; every row must be the table row at the oracle's index
+    w = W.CONFIGS[name]
+    p = device_params(w)
+    layer = EngramLayer.from_params(p)
+    ws = layer.workspace(w.B, w.T)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    layer.forward(p.ids, p.hidden, ws=ws, dev_status=st)
+    assert L.engram_read_status(st) == 0
+    idx = O.ngram_hash(oracle_ids(p), w.orders, w.heads_per_order, p.mult, p.primes, w.pad_id)
+    rows = torch.from_numpy(idx + np.asarray(p.offsets)[None, None, :]).to(DEV).view(-1)
+    M, E = w.B * w.T, w.nh * w.row_dim
+    expect = p.table[rows].view(M, E)
+    e = ws[: M * E * p.table.element_size()].view(p.table.dtype).view(M, E)
+    assert torch.equal(e, expect)
 
 
 def test_forward_zero_conv_is_gated_value():
