@@ -8,10 +8,12 @@
 //                                                     formulas §3.2; explainer §2.2 3)
 //
 // The conv is memory-bound: it reads V once (plus a (K-1)*dil halo per tile)
-// and writes hc times as many Y bytes.  Each thread owns two adjacent channels
-// (one 4-byte bf16x2 or 8-byte float2 access, coalesced across the warp) of
-// one sequence tile; the K taps of a position are re-read from L1, the gates
-// are warp-uniform broadcast loads.
+// and writes hc times as many Y bytes; U = g*V is formed on the fly and never
+// stored.  Forms, by shape: the tile form (V rows staged in shared memory,
+// bf16, K = 4, 256-channel slices), the run form (register windows along a
+// residue class; fp32 or other widths), the flat form (one thread per
+// position and 8 channels; short chunks and other tap counts) and the decode
+// step (T = 1 with the streaming state, which it also advances).
 #include "engram_internal.cuh"
 
 namespace engram {
@@ -364,8 +366,9 @@ __global__ void __launch_bounds__(kConvThreads) conv_run_kernel(const __grid_con
 }
 
 // Tile form for K = 4 taps, bfloat16, 256-channel slices.  A block owns
-// tile_t (32 to 64) consecutive positions of one sequence and one 256-channel slice, all
-// branches (one warp per branch, 8 channels per lane).  It first copies the V
+// tile_t (32 to 64) consecutive positions of one sequence and one 256-channel
+// slice, all branches (one warp per branch, 8 channels per lane).  It first
+// copies the V
 // rows of the tile and of its 3*dil-row halo into shared memory with cp.async
 // (one 16-byte piece per request, no registers held; halo rows before the
 // chunk come from the state ring or are zero) and their gates, then every
