@@ -429,6 +429,88 @@ def run_e2e(args, layer, p, w, device, world):
             "overlap": "copies of neighbouring steps overlap the forward (3 streams, 2 buffers)"}
 
 
+def run_offload(args, layer, p, w, device):
+    """Tables resident in pinned host memory (explainer §4.4), prefill
+    workloads: the same steps as the headline loop (L2 flushed between steps)
+    with (a) the device-resident table, (b) the host-resident table read by
+    the forward's gather over the host link, and (c) the pages' hash-ahead
+    form: engram_gather_ids for step i+1 on a second stream (host table) while
+    engram_forward_gathered runs step i, two row buffers."""
+    from hashed_gram_conditional_hash_b200 import EngramLayer
+    host_tab = p.table.cpu().pin_memory()
+    hl = EngramLayer(orders=w.orders, heads_per_order=w.heads_per_order, row_dim=w.row_dim,
+                     hidden=w.hidden, hc_mult=w.hc_mult, conv_kernel=w.conv_kernel,
+                     dilation=w.dil, pad_id=w.pad_id, vocab=w.vocab, table=host_tab,
+                     row_offsets=p.offsets, primes=p.primes, multipliers=p.mult,
+                     w_value=p.w_value, w_key=p.w_key, norm_key=p.norm_key,
+                     norm_query=p.norm_query, conv_w=p.conv_w, lookup=p.lookup,
+                     rms_eps=w.rms_eps, gate_eps=w.gate_eps)
+    B, T = w.B, w.T
+    ws = layer.workspace(B, T)
+    y = torch.empty((B, T, w.hc_mult, w.hidden), dtype=w.torch_dtype, device=device)
+    e = [hl.gather_ids(p.ids) for _ in range(2)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    comp = torch.cuda.current_stream()
+    side = torch.cuda.Stream(device=device)
+    ready, free = [torch.cuda.Event(), torch.cuda.Event()], [torch.cuda.Event(), torch.cuda.Event()]
+    for ev in free:
+        ev.record(comp)
+    K = max(3, min(args.steps, 200))
+
+    def timed(step):
+        for i in range(3):
+            step(i)
+            flush.fill_(i & 0xff)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        side.wait_event(e0)
+        for i in range(K):
+            step(i)
+            flush.fill_(i & 0xff)
+        comp.wait_stream(side)
+        e1.record(comp)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K          # ms per step, flushes included
+
+    def flush_ms():
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(comp)
+        for i in range(K):
+            flush.fill_(i & 0xff)
+        e1.record(comp)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K
+
+    def ahead(i):
+        b = i & 1
+        # rows of step i + 1 on the side stream (host table) ...
+        side.wait_event(free[(i + 1) & 1])
+        with torch.cuda.stream(side):
+            hl.gather_ids(p.ids, e=e[(i + 1) & 1])
+            ready[(i + 1) & 1].record(side)
+        # ... while step i runs on rows gathered one step earlier
+        if i > 0:                                  # (step 0's rows were gathered before the loop)
+            comp.wait_event(ready[b])
+        layer.forward_gathered(e[b], p.hidden, y=y, ws=ws)
+        free[b].record(comp)
+
+    f = flush_ms()
+    t_dev = timed(lambda i: layer.forward(p.ids, p.hidden, y=y, ws=ws)) - f
+    t_host = timed(lambda i: hl.forward(p.ids, p.hidden, y=y, ws=ws)) - f
+    t_ahead = timed(ahead) - f
+    tok = B * T
+    rows_mb = tok * w.nh * w.row_dim * p.table.element_size() / 1e6
+    from hashed_gram_conditional_hash_b200 import workloads as W
+    return {"table_gb": round(W.table_bytes(w) / 1e9, 3), "rows_per_step_mb": round(rows_mb, 1),
+            "device_table_tokens_per_s": tok / (t_dev / 1e3),
+            "host_table_tokens_per_s": tok / (t_host / 1e3),
+            "host_table_hash_ahead_tokens_per_s": tok / (t_ahead / 1e3),
+            "cost_host_table": 1.0 - t_dev / t_host, "cost_hash_ahead": 1.0 - t_dev / t_ahead,
+            "note": "step times exclude the L2 flush between steps; one Engram layer, no other "
+                    "layers' compute to hide the host-link transfer behind"}
+
+
 def run_reference(args):
     """The reference arm: the float64 oracle on the host cores, K timed steps
     of a bounded sample each, sized so that warm-up + steps take ~2 minutes."""
@@ -471,6 +553,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--decode-calls", type=int, default=0,
                     help="decode workload: number of distinct calls drawn (default: all 256)")
+    ap.add_argument("--offload", action="store_true",
+                    help="also measure tables resident in pinned host memory (prefill workloads)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -492,6 +576,8 @@ def main():
         res, layer, p, w = run_ours(args, rank, world, device)
         if not args.no_e2e:
             res["e2e"] = run_e2e(args, layer, p, w, device, world)
+        if args.offload and not w.decode_calls:
+            res["offload"] = run_offload(args, layer, p, w, device)
         del layer, p
         torch.cuda.empty_cache()
         if rank == 0 and not args.no_cpu_baseline and world == 1:

@@ -95,6 +95,9 @@ def lib() -> C.CDLL:
                                          C.POINTER(EngramState), P, sz, P, P]),
             "engram_forward_no_alloc": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P,
                                                   P, C.POINTER(EngramState), P, P]),
+            "engram_gather_ids": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P, P, P, P]),
+            "engram_forward_gathered": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P, P, P, sz,
+                                                  P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -275,6 +278,21 @@ def engram_forward(cfg: EngramConfig, weights: EngramWeights, ids: torch.Tensor,
     _check(lib().engram_forward(C.byref(cfg), C.byref(weights), _ptr(ids), B, T, _ptr(hidden),
                                 _ptr(y), C.byref(state) if state is not None else None, _ptr(ws),
                                 ws.numel(), _ptr(dev_status), _stream(stream)))
+
+
+def engram_gather_ids(cfg: EngramConfig, weights: EngramWeights, ids: torch.Tensor, e: torch.Tensor,
+                      history: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+                      stream=None) -> None:
+    B, T = ids.shape
+    _check(lib().engram_gather_ids(C.byref(cfg), C.byref(weights), _ptr(ids), B, T, _ptr(history), _ptr(e),
+                                   _ptr(dev_status), _stream(stream)))
+
+
+def engram_forward_gathered(cfg: EngramConfig, weights: EngramWeights, e: torch.Tensor, B: int, T: int,
+                            hidden: torch.Tensor, y: torch.Tensor, ws: torch.Tensor,
+                            dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(lib().engram_forward_gathered(C.byref(cfg), C.byref(weights), _ptr(e), B, T, _ptr(hidden), _ptr(y),
+                                         _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
 
 
 NO_ALLOC_SCRATCH_BYTES = 32 << 20

@@ -37,6 +37,28 @@ engram_status cuda_check(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Where the table lives: device (or managed) memory, or pinned host memory
+// the GPU reads over the host link (its device address in *dev).  Pageable
+// host memory is rejected: the GPU cannot read it.
+engram_status table_location(const void* table, const void** dev, bool* host) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, table) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(ENGRAM_ERR_INVALID_ARG, "table: not a CUDA-visible pointer");
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+    *dev = table;
+    *host = false;
+    return ENGRAM_OK;
+  }
+  if (a.type == cudaMemoryTypeHost && a.devicePointer != nullptr) {
+    *dev = a.devicePointer;
+    *host = true;
+    return ENGRAM_OK;
+  }
+  return fail(ENGRAM_ERR_INVALID_ARG, "table must be device memory or pinned (page-locked) host memory");
+}
+
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 int max_order(const engram_config& c) {
@@ -189,6 +211,101 @@ engram_status run_stage(const engram_config* c, ProjParams pp, float* g, float* 
   gp.rms_eps = c->rms_eps;
   gp.gate_eps = c->gate_eps;
   return cuda_check(launch_gate(gp, s), "gate");
+}
+
+// Everything after the row gather (a5-a9 and the state advance), on a dense
+// e (rows == null; a_src = e [M, E]) or, for the fused-gather path, on the
+// table with the head-major absolute rows (a_src = table).  Shared by
+// engram_forward and engram_forward_gathered.
+engram_status forward_tail(const engram_config* cfg, const engram_weights* wts, const ForwardLayout& L,
+                           char* w, const void* a_src, const int32_t* rows, int64_t ld, const float* wprod,
+                           int nh, int n_hist, const int64_t* ids, int32_t B, int32_t T, const void* hidden,
+                           void* y, const engram_state* state, uint32_t* dev_status, cudaStream_t s) {
+  engram_status st = ENGRAM_OK;
+  const int64_t M = static_cast<int64_t>(B) * T;
+  // a5-a7: projection, score partials, gates
+  ProjParams pp;
+  memset(&pp, 0, sizeof pp);
+  pp.a_src = a_src;
+  pp.rows = rows;
+  pp.ld_rows = ld;
+  pp.a_rows = rows != nullptr ? wts->total_rows : M * nh;
+  pp.w_value = wts->w_value;
+  pp.w_key = wts->w_key;
+  pp.norm_key = wts->norm_key;
+  pp.norm_query = wts->norm_query;
+  pp.hidden = hidden;
+  pp.V = w + L.st.v_off;
+  pp.partials = reinterpret_cast<float4*>(w + L.st.part_off);
+  pp.wprod = wprod;
+  pp.status = dev_status;
+  pp.M = M;
+  pp.nh = nh;
+  pp.Dh = cfg->row_dim;
+  pp.E = nh * cfg->row_dim;
+  pp.H = cfg->hidden;
+  pp.hc = cfg->hc_mult;
+  pp.dtype = cfg->dtype;
+  float* g = reinterpret_cast<float*>(w + L.st.g_off);
+
+  // a8-a9: gated value, short conv, residual
+  ConvParams cp;
+  memset(&cp, 0, sizeof cp);
+  cp.V = pp.V;
+  cp.g = g;
+  cp.conv_w = wts->conv_w;
+  cp.Y = y;
+  if (state != nullptr) {
+    cp.v_ring = state->v_ring;
+    cp.g_ring = state->g_ring;
+    cp.pos = state->pos;
+    cp.pos_lag = T;  // advanced by the gate kernel
+    cp.ring_len = state->ring_len;
+  }
+  cp.B = B;
+  cp.T = T;
+  cp.H = cfg->hidden;
+  cp.hc = cfg->hc_mult;
+  cp.K = cfg->conv_kernel;
+  cp.dil = cfg->dilation;
+  cp.dtype = cfg->dtype;
+  // with the streaming state the gate kernel also takes the chunk's ids into
+  // the id ring (the hash has read it) and advances pos (the conv reads pos - T)
+  StateIdsAdvance sa;
+  memset(&sa, 0, sizeof sa);
+  if (state != nullptr) {
+    sa.id_ring = state->id_ring;
+    sa.pos = state->pos;
+    sa.ids = ids;
+    sa.lookup = wts->lookup;
+    sa.status = dev_status;
+    sa.raw_vocab = wts->raw_vocab;
+    sa.vocab = cfg->vocab;
+    sa.pad_id = cfg->pad_id;
+    sa.B = B;
+    sa.T = T;
+    sa.n_hist = n_hist;
+  }
+  st = run_stage(cfg, pp, g, nullptr, s, state != nullptr ? &sa : nullptr);
+  if (st != ENGRAM_OK) return st;
+  record(g_events.before_conv, s);
+  st = cuda_check(launch_gated_conv(cp, s), "gated conv");
+  record(g_events.after_conv, s);
+  if (st != ENGRAM_OK || state == nullptr || conv_writes_rings(cp)) return st;
+
+  StateAdvanceParams ap;
+  ap.V = pp.V;
+  ap.g = g;
+  ap.v_ring = state->v_ring;
+  ap.g_ring = state->g_ring;
+  ap.pos = state->pos;
+  ap.ring_len = state->ring_len;
+  ap.B = B;
+  ap.T = T;
+  ap.H = cfg->hidden;
+  ap.hc = cfg->hc_mult;
+  ap.dtype = cfg->dtype;
+  return cuda_check(launch_state_advance(ap, s), "state advance");
 }
 
 }  // namespace
@@ -504,7 +621,15 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   // rows for the fused-gather path (rows with a width that is not a multiple
   // of 16 bytes also take that path: the projection gathers them itself)
   const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
-  const bool fused = (g_debug.load() & ENGRAM_DEBUG_FUSED_GATHER) != 0 || (row_bytes % 16) != 0;
+  const void* table = nullptr;
+  bool table_host = false;
+  st = table_location(wts->table, &table, &table_host);
+  if (st != ENGRAM_OK) return st;
+  if (table_host && row_bytes % 16 != 0)
+    return fail(ENGRAM_ERR_UNSUPPORTED, "a host-resident table needs rows of a multiple of 16 bytes");
+  // a host-resident table is read only by the gather kernel (never by the projection's TMA)
+  const bool fused = !table_host &&
+                     ((g_debug.load() & ENGRAM_DEBUG_FUSED_GATHER) != 0 || (row_bytes % 16) != 0);
   const int64_t ld = rows_ld(M);
   int32_t* rows = reinterpret_cast<int32_t*>(w + L.rows_off);
   void* e = w + L.e_off;
@@ -524,7 +649,8 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   } else {
     HashGatherParams hg;
     hg.h = hp;
-    hg.table = wts->table;
+    hg.table = table;
+    hg.table_host = table_host ? 1 : 0;
     hg.e = e;
     hg.row_bytes = row_bytes;
     // the score's RMSNorm weight products, once per call, for the projection
@@ -536,89 +662,85 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   }
   if (st != ENGRAM_OK) return st;
 
-  // a5-a7: projection, score partials, gates
-  ProjParams pp;
-  memset(&pp, 0, sizeof pp);
-  pp.a_src = fused ? wts->table : e;
-  pp.rows = fused ? rows : nullptr;
-  pp.ld_rows = ld;
-  pp.a_rows = fused ? wts->total_rows : M * hp.nh;
-  pp.w_value = wts->w_value;
-  pp.w_key = wts->w_key;
-  pp.norm_key = wts->norm_key;
-  pp.norm_query = wts->norm_query;
-  pp.hidden = hidden;
-  pp.V = w + L.st.v_off;
-  pp.partials = reinterpret_cast<float4*>(w + L.st.part_off);
-  pp.wprod = (!fused && cfg->dtype == ENGRAM_BF16) ? reinterpret_cast<const float*>(w + L.wp_off) : nullptr;
-  pp.status = dev_status;
-  pp.M = M;
-  pp.nh = hp.nh;
-  pp.Dh = cfg->row_dim;
-  pp.E = hp.nh * cfg->row_dim;
-  pp.H = cfg->hidden;
-  pp.hc = cfg->hc_mult;
-  pp.dtype = cfg->dtype;
-  float* g = reinterpret_cast<float*>(w + L.st.g_off);
+  return forward_tail(cfg, wts, L, w, fused ? wts->table : e, fused ? rows : nullptr, ld,
+                      (!fused && cfg->dtype == ENGRAM_BF16) ? reinterpret_cast<const float*>(w + L.wp_off) : nullptr,
+                      hp.nh, hp.n_hist, ids, B, T, hidden, y, state, dev_status, s);
+}
 
-  // a8-a9: gated value, short conv, residual
-  ConvParams cp;
-  memset(&cp, 0, sizeof cp);
-  cp.V = pp.V;
-  cp.g = g;
-  cp.conv_w = wts->conv_w;
-  cp.Y = y;
-  if (state != nullptr) {
-    cp.v_ring = state->v_ring;
-    cp.g_ring = state->g_ring;
-    cp.pos = state->pos;
-    cp.pos_lag = T;  // advanced by the gate kernel
-    cp.ring_len = state->ring_len;
-  }
-  cp.B = B;
-  cp.T = T;
-  cp.H = cfg->hidden;
-  cp.hc = cfg->hc_mult;
-  cp.K = cfg->conv_kernel;
-  cp.dil = cfg->dilation;
-  cp.dtype = cfg->dtype;
-  // with the streaming state the gate kernel also takes the chunk's ids into
-  // the id ring (the hash has read it) and advances pos (the conv reads pos - T)
-  StateIdsAdvance sa;
-  memset(&sa, 0, sizeof sa);
-  if (state != nullptr) {
-    sa.id_ring = state->id_ring;
-    sa.pos = state->pos;
-    sa.ids = ids;
-    sa.lookup = wts->lookup;
-    sa.status = dev_status;
-    sa.raw_vocab = wts->raw_vocab;
-    sa.vocab = cfg->vocab;
-    sa.pad_id = cfg->pad_id;
-    sa.B = B;
-    sa.T = T;
-    sa.n_hist = hp.n_hist;
-  }
-  st = run_stage(cfg, pp, g, nullptr, s, state != nullptr ? &sa : nullptr);
+engram_status engram_gather_ids(const engram_config* cfg, const engram_weights* wts, const int64_t* ids,
+                                int32_t B, int32_t T, const int64_t* history, void* e, uint32_t* dev_status,
+                                engram_stream stream) {
+  engram_status st = check_config(cfg);
   if (st != ENGRAM_OK) return st;
-  record(g_events.before_conv, s);
-  st = cuda_check(launch_gated_conv(cp, s), "gated conv");
-  record(g_events.after_conv, s);
-  if (st != ENGRAM_OK || state == nullptr || conv_writes_rings(cp)) return st;
+  if (wts == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights is NULL");
+  if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
+  const int64_t M = static_cast<int64_t>(B) * T;
+  if (M == 0) return ENGRAM_OK;
+  const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
+  if (row_bytes % 16 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
+  if (wts->table == nullptr || ids == nullptr || e == nullptr)
+    return fail(ENGRAM_ERR_INVALID_ARG, "table / ids / e must be non-NULL");
+  if (!aligned16(e) || !aligned16(ids)) return fail(ENGRAM_ERR_INVALID_ARG, "ids and e must be 16-byte aligned");
+  if (wts->row_offsets == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "row_offsets (host) is NULL");
+  if (wts->lookup != nullptr && wts->raw_vocab < 1) return fail(ENGRAM_ERR_INVALID_ARG, "raw_vocab < 1");
+  if (wts->total_rows < 1 || wts->total_rows > INT32_MAX)
+    return fail(ENGRAM_ERR_UNSUPPORTED, "total_rows must be in [1, 2^31)");
+  const void* table = nullptr;
+  bool table_host = false;
+  st = table_location(wts->table, &table, &table_host);
+  if (st != ENGRAM_OK) return st;
+  if (!table_host && !aligned16(table)) return fail(ENGRAM_ERR_INVALID_ARG, "table must be 16-byte aligned");
+  HashParams hp;
+  st = fill_hash_params(cfg, wts->multipliers, wts->primes, &hp);
+  if (st != ENGRAM_OK) return st;
+  for (int h = 0; h < hp.nh; ++h) {
+    const int64_t off = wts->row_offsets[h];
+    if (off < 0 || off + wts->primes[h] > wts->total_rows)
+      return fail(ENGRAM_ERR_INVALID_ARG, "table %d (rows [%lld, %lld)) exceeds total_rows", h,
+                  static_cast<long long>(off), static_cast<long long>(off + wts->primes[h]));
+    hp.row_off[h] = off;
+  }
+  hp.ids = ids;
+  hp.lookup = wts->lookup;
+  hp.raw_vocab = wts->raw_vocab;
+  hp.history = history;
+  hp.status = dev_status;
+  hp.B = B;
+  hp.T = T;
+  HashGatherParams hg;
+  memset(&hg, 0, sizeof hg);
+  hg.h = hp;
+  hg.table = table;
+  hg.table_host = table_host ? 1 : 0;
+  hg.e = e;
+  hg.row_bytes = row_bytes;
+  return cuda_check(launch_hash_gather(hg, static_cast<cudaStream_t>(stream)), "hash+gather");
+}
 
-  StateAdvanceParams ap;
-  ap.V = pp.V;
-  ap.g = g;
-  ap.v_ring = state->v_ring;
-  ap.g_ring = state->g_ring;
-  ap.pos = state->pos;
-  ap.ring_len = state->ring_len;
-  ap.B = B;
-  ap.T = T;
-  ap.H = cfg->hidden;
-  ap.hc = cfg->hc_mult;
-  ap.dtype = cfg->dtype;
-  return cuda_check(launch_state_advance(ap, s), "state advance");
+engram_status engram_forward_gathered(const engram_config* cfg, const engram_weights* wts, const void* e,
+                                      int32_t B, int32_t T, const void* hidden, void* y, void* ws,
+                                      size_t ws_bytes, uint32_t* dev_status, engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  st = check_dense_shapes(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (wts == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights is NULL");
+  if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
+  const int64_t M = static_cast<int64_t>(B) * T;
+  if (M == 0) return ENGRAM_OK;
+  const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
+  if (row_bytes % 16 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
+  const void* ptrs[] = {e, wts->w_value, wts->w_key, wts->norm_key, wts->norm_query, wts->conv_w, hidden, y, ws};
+  for (const void* p : ptrs) {
+    if (p == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "a tensor / workspace pointer is NULL");
+    if (!aligned16(p)) return fail(ENGRAM_ERR_INVALID_ARG, "tensor / workspace pointers must be 16-byte aligned");
+  }
+  const ForwardLayout L = forward_layout(cfg, M);
+  if (ws_bytes < L.end)
+    return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", ws_bytes, L.end);
+  const int nh = cfg->n_orders * cfg->heads_per_order;
+  return forward_tail(cfg, wts, L, static_cast<char*>(ws), e, nullptr, rows_ld(M), nullptr, nh, 0, nullptr, B, T,
+                      hidden, y, nullptr, dev_status, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

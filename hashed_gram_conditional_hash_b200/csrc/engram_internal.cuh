@@ -66,6 +66,7 @@ struct HashGatherParams {
   const void* table;
   void* e;                  // [B*T, nh*Dh]
   int32_t row_bytes;
+  int32_t table_host;       // 1: the table is pinned host memory (read over the host link)
   FastDiv div_nh, div_J, div_T;   // set by launch_hash_gather
   // optional side job for the projection that follows: wprod[i] = nk[i] * nq[i]
   const uint16_t* nk;

@@ -117,12 +117,17 @@ __device__ __forceinline__ int64_t hashed_row(const HashGatherParams& g, int q) 
   return p.row_off[h] + static_cast<int64_t>(barrett_mod(mix, p.prime[h], p.barrett[h]));
 }
 
-// A 16-byte piece of a table row: read once, so it bypasses L1.
+// A 16-byte piece of a table row: read once, so it bypasses L1.  A table in
+// pinned host memory is read with plain loads (over the host link).
+template <bool HOSTMEM>
 __device__ __forceinline__ int4 ld_row_piece(const int4* p) {
   int4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.s32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
+  if (HOSTMEM)
+    asm volatile("ld.global.v4.s32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  else
+    asm volatile("ld.global.nc.L1::no_allocate.v4.s32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
   return v;
 }
 
@@ -132,7 +137,7 @@ __device__ __forceinline__ int4 ld_row_piece(const int4* p) {
 // known at compile time (8: 64 bf16), else 0 (read from the params; ROWS 32).
 // Fewer rows per warp means more warps, each with one short dependent chain
 // (ids -> hash -> rows -> e), which is what the random row reads want.
-template <int CH, int ROWS>
+template <int CH, int ROWS, bool HOSTMEM>
 __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant__ HashGatherParams g) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const HashParams& p = g.h;
@@ -157,7 +162,8 @@ __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant_
       const int i = u * 32 + lane;
       const int r = i / CH;
       const int64_t src = __shfl_sync(0xffffffffu, row, r);
-      if (q0 + r < total) v[u] = ld_row_piece(reinterpret_cast<const int4*>(tab + src * (CH * 16)) + (i - r * CH));
+      if (q0 + r < total)
+        v[u] = ld_row_piece<HOSTMEM>(reinterpret_cast<const int4*>(tab + src * (CH * 16)) + (i - r * CH));
     }
     int4* out = static_cast<int4*>(g.e) + static_cast<int64_t>(q0) * CH;
 #pragma unroll
@@ -179,7 +185,7 @@ __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant_
       const int r = i / chunks;
       const int64_t src = __shfl_sync(0xffffffffu, row, r % ROWS);
       if (i < per && q0 + r < total)
-        v[u] = __ldg(reinterpret_cast<const int4*>(tab + src * g.row_bytes) + (i - r * chunks));
+        v[u] = ld_row_piece<HOSTMEM>(reinterpret_cast<const int4*>(tab + src * g.row_bytes) + (i - r * chunks));
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -230,10 +236,16 @@ cudaError_t launch_hash_gather(const HashGatherParams& g0, cudaStream_t s) {
     if (total * (32 / kRows) + 256 > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit ids in the kernel
     if (g.row_bytes == 128) {
       const int64_t blocks = (total + 8 * kRows - 1) / (8 * kRows);
-      launch_k(hash_gather_kernel<8, kRows>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
+      if (g.table_host)
+        launch_k(hash_gather_kernel<8, kRows, true>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
+      else
+        launch_k(hash_gather_kernel<8, kRows, false>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
     } else {
       const int64_t blocks = (total + 255) / 256;
-      launch_k(hash_gather_kernel<0, 32>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
+      if (g.table_host)
+        launch_k(hash_gather_kernel<0, 32, true>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
+      else
+        launch_k(hash_gather_kernel<0, 32, false>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

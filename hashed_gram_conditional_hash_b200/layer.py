@@ -39,6 +39,13 @@ class EngramLayer:
         self._host = [np.ascontiguousarray(np.asarray(a, dtype=np.int64))
                       for a in (row_offsets, primes, multipliers)]
         self._dev = [table, w_value, w_key, norm_key, norm_query, conv_w, lookup]
+        # the table may live in pinned host memory (read over the host link);
+        # everything else, and every workspace, lives on the weights' device
+        self.device = w_value.device
+        if table.device.type == "cpu" and not table.is_pinned():
+            raise ValueError("a host-resident table must be in pinned memory (tensor.pin_memory())")
+        self.row_width = table.shape[1]
+        self.nh = len(primes)
         for t in self._dev:
             if t is not None and not t.is_contiguous():
                 raise ValueError("layer tensors must be contiguous")
@@ -72,10 +79,10 @@ class EngramLayer:
     def workspace(self, B: int, T: int, device=None) -> torch.Tensor:
         n = L.engram_forward_workspace_size(self.cfg, B, T)
         return torch.empty(max(n, 256), dtype=torch.uint8,
-                           device=device or self._dev[0].device)
+                           device=device or self.device)
 
     def new_state(self, B: int, stream=None) -> StreamState:
-        dev = self._dev[0].device
+        dev = self.device
         id_ring = torch.empty((B, max(self.max_n - 1, 1)), dtype=torch.int64, device=dev)
         v_ring = torch.empty((B, self.ring_len, self.hidden), dtype=self.dtype, device=dev)
         g_ring = torch.empty((B, self.ring_len, self.hc), dtype=torch.float32, device=dev)
@@ -88,6 +95,28 @@ class EngramLayer:
         c.ring_len = self.ring_len
         L.engram_state_init(self.cfg, c, B, stream)
         return StreamState(c, id_ring, v_ring, g_ring, pos)
+
+    def gather_ids(self, ids: torch.Tensor, e: Optional[torch.Tensor] = None,
+                   history: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+        """The gathered rows e [B*T, nh*Dh] of ids (engram_gather_ids)."""
+        B, T = ids.shape
+        if e is None:
+            e = torch.empty((B * T, self.nh * self.row_width), dtype=self.dtype, device=ids.device)
+        L.engram_gather_ids(self.cfg, self.weights, ids, e, history, dev_status, stream)
+        return e
+
+    def forward_gathered(self, e: torch.Tensor, hidden: torch.Tensor, y: Optional[torch.Tensor] = None,
+                         ws: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+        """The pass on rows from gather_ids (engram_forward_gathered), no state."""
+        B, T = hidden.shape[0], hidden.shape[1]
+        if y is None:
+            y = torch.empty((B, T, self.hc, self.hidden), dtype=self.dtype, device=hidden.device)
+        if ws is None:
+            ws = self.workspace(B, T, hidden.device)
+        L.engram_forward_gathered(self.cfg, self.weights, e, B, T, hidden, y, ws, dev_status, stream)
+        return y
 
     def forward(self, ids: torch.Tensor, hidden: torch.Tensor, y: Optional[torch.Tensor] = None,
                 ws: Optional[torch.Tensor] = None, state: Optional[StreamState] = None,

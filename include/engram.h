@@ -241,7 +241,8 @@ engram_status engram_state_init(const engram_config* cfg, const engram_state* st
                                 engram_stream stream);
 
 /* Engram.forward(hidden_states, input_ids) of the explainer page §4.3, all steps
- * a1-a9 on the device.
+ * a1-a9 on the device.  weights->table may be device memory or pinned host
+ * memory (read over the host link by the gather; see engram_gather_ids).
  *   ids:    DEVICE int64 [B, T]; raw ids when weights->lookup is set, else compressed
  *   hidden: DEVICE [B, T, hc, H];  y: DEVICE [B, T, hc, H]
  *   state:  NULL for an independent prefill; otherwise the sequences continue
@@ -256,6 +257,38 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wei
                              const int64_t* ids, int32_t B, int32_t T, const void* hidden,
                              void* y, const engram_state* state, void* ws, size_t ws_bytes,
                              uint32_t* dev_status, engram_stream stream);
+
+/* ---- the pass in two halves: gather ahead, then compute ---------------- */
+
+/* Hash-ahead gather (explainer §4.4: the indices depend only on the ids, so
+ * the rows can be fetched before the layer runs): a1-a4 of engram_forward in
+ * one kernel, into a caller buffer.
+ *   e[m, (o*J + j)*Dh + c] = table[row_offsets[o*J+j] + idx[m, o*J+j], c]
+ * ids: DEVICE int64 [B, T] (raw when weights->lookup is set); history: DEVICE
+ * [B, max_order-1] ids before the chunk (most recent last) or NULL (pad_id);
+ * e: DEVICE [B*T, nh*Dh] in dtype, 16-byte aligned.  Uses weights->table,
+ * total_rows, row_offsets, primes, multipliers, lookup, raw_vocab.
+ * weights->table may be device memory or PINNED host memory (cudaHostAlloc /
+ * cudaHostRegister): host rows are read over the host link, so a caller can
+ * keep tables larger than HBM on the host and run this call on a second
+ * stream one chunk ahead of engram_forward_gathered.  Pageable host memory is
+ * rejected (ENGRAM_ERR_INVALID_ARG).  Rows must be a multiple of 16 bytes
+ * (ENGRAM_ERR_UNSUPPORTED otherwise).  Out-of-range ids set
+ * ENGRAM_STATUS_ID_RANGE and hash as pad_id. */
+engram_status engram_gather_ids(const engram_config* cfg, const engram_weights* weights, const int64_t* ids,
+                                int32_t B, int32_t T, const int64_t* history, void* e, uint32_t* dev_status,
+                                engram_stream stream);
+
+/* The rest of engram_forward (a5-a9) on rows gathered by engram_gather_ids:
+ * y = the same result engram_forward gives for those ids (bit for bit on the
+ * same engine), without the streaming state (independent sequences or a
+ * caller that keeps no state).  e: DEVICE [B*T, nh*Dh]; hidden, y: DEVICE
+ * [B, T, hc, H]; ws: DEVICE scratch of engram_forward_workspace_size(cfg, B, T)
+ * bytes, 256-byte aligned.  Uses weights->w_value, w_key, norm_key,
+ * norm_query, conv_w. */
+engram_status engram_forward_gathered(const engram_config* cfg, const engram_weights* weights, const void* e,
+                                      int32_t B, int32_t T, const void* hidden, void* y, void* ws,
+                                      size_t ws_bytes, uint32_t* dev_status, engram_stream stream);
 
 /* ---- the whole pass without caller scratch ----------------------------- */
 

@@ -1,0 +1,93 @@
+"""The pass in two halves (engram_gather_ids, then engram_forward_gathered)
+and tables resident in pinned host memory (explainer §4.4: the indices depend
+only on the ids, so rows can be fetched ahead of the layer, from host RAM).
+
+The halves must give engram_forward's result bit for bit, and a host-resident
+table the device-resident result bit for bit (the same rows reach the same
+kernels); pageable host memory is refused without a launch."""
+import numpy as np
+import pytest
+import torch
+
+from hashed_gram_conditional_hash_b200 import EngramLayer
+from hashed_gram_conditional_hash_b200 import _lib as L
+from hashed_gram_conditional_hash_b200 import workloads as W
+
+from gpu_helpers import device_params, oracle_ids
+from oracle import engram_oracle as O
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _layer(p, table=None):
+    w = p.w
+    return EngramLayer(orders=w.orders, heads_per_order=w.heads_per_order, row_dim=w.row_dim,
+                       hidden=w.hidden, hc_mult=w.hc_mult, conv_kernel=w.conv_kernel,
+                       dilation=w.dil, pad_id=w.pad_id, vocab=w.vocab,
+                       table=p.table if table is None else table, row_offsets=p.offsets,
+                       primes=p.primes, multipliers=p.mult, w_value=p.w_value, w_key=p.w_key,
+                       norm_key=p.norm_key, norm_query=p.norm_query, conv_w=p.conv_w,
+                       lookup=p.lookup, rms_eps=w.rms_eps, gate_eps=w.gate_eps)
+
+
+CASES = [W.small_workload(), W.small_workload(B=2, T=130, hidden=512, hc_mult=4, orders=(2, 3, 4)),
+         W.small_workload(B=2, T=60, raw_vocab=6500), W.small_workload(dtype="f32", B=2, T=50, row_dim=32,
+                                                                       hidden=128, hc_mult=3),
+         W.CONFIGS["model_bf16"]]
+
+
+@pytest.mark.parametrize("w", CASES, ids=[str(i) for i in range(len(CASES))])
+def test_gathered_halves_equal_forward(w):
+    p = device_params(w)
+    layer = _layer(p)
+    y = layer.forward(p.ids, p.hidden)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    e = layer.gather_ids(p.ids, dev_status=st)
+    y2 = layer.forward_gathered(e, p.hidden, dev_status=st)
+    assert L.engram_read_status(st) == 0
+    assert torch.equal(y, y2)
+    # the rows are the table rows at the oracle's indices
+    idx = O.ngram_hash(oracle_ids(p), w.orders, w.heads_per_order, p.mult, p.primes, w.pad_id)
+    rows = torch.from_numpy(idx + np.asarray(p.offsets)[None, None, :]).to(DEV).view(-1)
+    assert torch.equal(e, p.table[rows].view(e.shape))
+
+
+@pytest.mark.parametrize("w", CASES, ids=[str(i) for i in range(len(CASES))])
+def test_host_resident_table_equals_device_table(w):
+    p = device_params(w)
+    dev_layer = _layer(p)
+    host_layer = _layer(p, table=p.table.cpu().pin_memory())
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    assert torch.equal(host_layer.gather_ids(p.ids, dev_status=st), dev_layer.gather_ids(p.ids))
+    assert torch.equal(host_layer.forward(p.ids, p.hidden, dev_status=st), dev_layer.forward(p.ids, p.hidden))
+    assert L.engram_read_status(st) == 0
+
+
+def test_gather_ids_with_history_continues_sequences():
+    w = W.small_workload(B=3, T=40, orders=(2, 3, 4))
+    p = device_params(w)
+    layer = _layer(p)
+    full = layer.gather_ids(p.ids)
+    hist = p.ids[:, 17:20].contiguous()               # the 3 ids before position 20
+    tail = layer.gather_ids(p.ids[:, 20:].contiguous(), history=hist)
+    E = w.nh * w.row_dim
+    assert torch.equal(tail.view(w.B, -1, E), full.view(w.B, w.T, E)[:, 20:])
+
+
+def test_pageable_host_table_is_refused_without_launch():
+    w = W.small_workload()
+    p = device_params(w)
+    with pytest.raises(ValueError):
+        _layer(p, table=p.table.cpu())                 # the binding refuses it up front
+    layer = _layer(p)
+    pageable = p.table.cpu()                          # ... and so does the library itself
+    layer.weights.table = pageable.data_ptr()
+    e = torch.empty((w.B * w.T, w.nh * w.row_dim), dtype=p.table.dtype, device=DEV)
+    before = L.engram_launch_count()
+    with pytest.raises(L.EngramError) as ei:
+        L.engram_gather_ids(layer.cfg, layer.weights, p.ids, e)
+    assert ei.value.code == 1 and "pinned" in str(ei.value)
+    with pytest.raises(L.EngramError):
+        layer.forward(p.ids, p.hidden)
+    assert L.engram_launch_count() == before
