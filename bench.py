@@ -495,6 +495,20 @@ def run_offload(args, layer, p, w, device):
         layer.forward_gathered(e[b], p.hidden, y=y, ws=ws)
         free[b].record(comp)
 
+    # two Engram layers' rows of the same ids (own multipliers; the same
+    # device table here): one batched launch vs two gathers
+    from hashed_gram_conditional_hash_b200 import _lib as L
+    l2 = EngramLayer(orders=w.orders, heads_per_order=w.heads_per_order, row_dim=w.row_dim,
+                     hidden=w.hidden, hc_mult=w.hc_mult, conv_kernel=w.conv_kernel,
+                     dilation=w.dil, pad_id=w.pad_id, vocab=w.vocab, table=p.table,
+                     row_offsets=p.offsets, primes=p.primes, multipliers=p.mult[::-1].copy(),
+                     w_value=p.w_value, w_key=p.w_key, norm_key=p.norm_key,
+                     norm_query=p.norm_query, conv_w=p.conv_w, lookup=p.lookup,
+                     rms_eps=w.rms_eps, gate_eps=w.gate_eps)
+    e2 = [torch.empty_like(e[0]), torch.empty_like(e[0])]
+    t_pair = timed(lambda i: (layer.gather_ids(p.ids, e=e2[0]), l2.gather_ids(p.ids, e=e2[1])))
+    t_batched = timed(lambda i: L.engram_gather_ids_layers(layer.cfg, [layer.weights, l2.weights], p.ids, e2))
+
     f = flush_ms()
     t_dev = timed(lambda i: layer.forward(p.ids, p.hidden, y=y, ws=ws)) - f
     t_host = timed(lambda i: hl.forward(p.ids, p.hidden, y=y, ws=ws)) - f
@@ -507,6 +521,7 @@ def run_offload(args, layer, p, w, device):
             "host_table_tokens_per_s": tok / (t_host / 1e3),
             "host_table_hash_ahead_tokens_per_s": tok / (t_ahead / 1e3),
             "cost_host_table": 1.0 - t_dev / t_host, "cost_hash_ahead": 1.0 - t_dev / t_ahead,
+            "two_layer_gather_us": {"separate": (t_pair - f) * 1e3, "one_launch": (t_batched - f) * 1e3},
             "note": "step times exclude the L2 flush between steps; one Engram layer, no other "
                     "layers' compute to hide the host-link transfer behind"}
 

@@ -98,6 +98,8 @@ def lib() -> C.CDLL:
             "engram_gather_ids": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P, P, P, P]),
             "engram_forward_gathered": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P, P, P, sz,
                                                   P, P]),
+            "engram_gather_ids_layers": (C.c_int, [cfg, C.POINTER(C.POINTER(EngramWeights)), i32, P, i32, i32,
+                                                   P, C.POINTER(P), P, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -286,6 +288,22 @@ def engram_gather_ids(cfg: EngramConfig, weights: EngramWeights, ids: torch.Tens
     B, T = ids.shape
     _check(lib().engram_gather_ids(C.byref(cfg), C.byref(weights), _ptr(ids), B, T, _ptr(history), _ptr(e),
                                    _ptr(dev_status), _stream(stream)))
+
+
+MAX_LAYERS = 4
+
+
+def engram_gather_ids_layers(cfg: EngramConfig, weights: Sequence[EngramWeights], ids: torch.Tensor,
+                             e: Sequence[torch.Tensor], history: Optional[torch.Tensor] = None,
+                             dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    if len(weights) != len(e):
+        raise ValueError("one output per layer")
+    B, T = ids.shape
+    n = len(weights)
+    wp = (C.POINTER(EngramWeights) * n)(*[C.pointer(w) for w in weights])
+    ep = (C.c_void_p * n)(*[_ptr(t).value for t in e])
+    _check(lib().engram_gather_ids_layers(C.byref(cfg), wp, n, _ptr(ids), B, T, _ptr(history), ep,
+                                          _ptr(dev_status), _stream(stream)))
 
 
 def engram_forward_gathered(cfg: EngramConfig, weights: EngramWeights, e: torch.Tensor, B: int, T: int,

@@ -213,6 +213,52 @@ engram_status run_stage(const engram_config* c, ProjParams pp, float* g, float* 
   return cuda_check(launch_gate(gp, s), "gate");
 }
 
+// Checks and fills the parameters of the hash + gather of one layer's rows
+// into e (engram_gather_ids and engram_gather_ids_layers); B*T > 0.
+engram_status prepare_gather(const engram_config* cfg, const engram_weights* wts, const int64_t* ids,
+                             int32_t B, int32_t T, const int64_t* history, void* e, uint32_t* dev_status,
+                             HashGatherParams* hg) {
+  if (wts == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights is NULL");
+  const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
+  if (row_bytes % 16 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
+  if (wts->table == nullptr || ids == nullptr || e == nullptr)
+    return fail(ENGRAM_ERR_INVALID_ARG, "table / ids / e must be non-NULL");
+  if (!aligned16(e) || !aligned16(ids)) return fail(ENGRAM_ERR_INVALID_ARG, "ids and e must be 16-byte aligned");
+  if (wts->row_offsets == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "row_offsets (host) is NULL");
+  if (wts->lookup != nullptr && wts->raw_vocab < 1) return fail(ENGRAM_ERR_INVALID_ARG, "raw_vocab < 1");
+  if (wts->total_rows < 1 || wts->total_rows > INT32_MAX)
+    return fail(ENGRAM_ERR_UNSUPPORTED, "total_rows must be in [1, 2^31)");
+  const void* table = nullptr;
+  bool table_host = false;
+  engram_status st = table_location(wts->table, &table, &table_host);
+  if (st != ENGRAM_OK) return st;
+  if (!aligned16(table)) return fail(ENGRAM_ERR_INVALID_ARG, "table must be 16-byte aligned");
+  HashParams hp;
+  st = fill_hash_params(cfg, wts->multipliers, wts->primes, &hp);
+  if (st != ENGRAM_OK) return st;
+  for (int h = 0; h < hp.nh; ++h) {
+    const int64_t off = wts->row_offsets[h];
+    if (off < 0 || off + wts->primes[h] > wts->total_rows)
+      return fail(ENGRAM_ERR_INVALID_ARG, "table %d (rows [%lld, %lld)) exceeds total_rows", h,
+                  static_cast<long long>(off), static_cast<long long>(off + wts->primes[h]));
+    hp.row_off[h] = off;
+  }
+  hp.ids = ids;
+  hp.lookup = wts->lookup;
+  hp.raw_vocab = wts->raw_vocab;
+  hp.history = history;
+  hp.status = dev_status;
+  hp.B = B;
+  hp.T = T;
+  memset(hg, 0, sizeof *hg);
+  hg->h = hp;
+  hg->table = table;
+  hg->table_host = table_host ? 1 : 0;
+  hg->e = e;
+  hg->row_bytes = row_bytes;
+  return ENGRAM_OK;
+}
+
 // Everything after the row gather (a5-a9 and the state advance), on a dense
 // e (rows == null; a_src = e [M, E]) or, for the fused-gather path, on the
 // table with the head-major absolute rows (a_src = table).  Shared by
@@ -672,49 +718,33 @@ engram_status engram_gather_ids(const engram_config* cfg, const engram_weights* 
                                 engram_stream stream) {
   engram_status st = check_config(cfg);
   if (st != ENGRAM_OK) return st;
-  if (wts == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights is NULL");
   if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
-  const int64_t M = static_cast<int64_t>(B) * T;
-  if (M == 0) return ENGRAM_OK;
-  const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
-  if (row_bytes % 16 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
-  if (wts->table == nullptr || ids == nullptr || e == nullptr)
-    return fail(ENGRAM_ERR_INVALID_ARG, "table / ids / e must be non-NULL");
-  if (!aligned16(e) || !aligned16(ids)) return fail(ENGRAM_ERR_INVALID_ARG, "ids and e must be 16-byte aligned");
-  if (wts->row_offsets == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "row_offsets (host) is NULL");
-  if (wts->lookup != nullptr && wts->raw_vocab < 1) return fail(ENGRAM_ERR_INVALID_ARG, "raw_vocab < 1");
-  if (wts->total_rows < 1 || wts->total_rows > INT32_MAX)
-    return fail(ENGRAM_ERR_UNSUPPORTED, "total_rows must be in [1, 2^31)");
-  const void* table = nullptr;
-  bool table_host = false;
-  st = table_location(wts->table, &table, &table_host);
-  if (st != ENGRAM_OK) return st;
-  if (!table_host && !aligned16(table)) return fail(ENGRAM_ERR_INVALID_ARG, "table must be 16-byte aligned");
-  HashParams hp;
-  st = fill_hash_params(cfg, wts->multipliers, wts->primes, &hp);
-  if (st != ENGRAM_OK) return st;
-  for (int h = 0; h < hp.nh; ++h) {
-    const int64_t off = wts->row_offsets[h];
-    if (off < 0 || off + wts->primes[h] > wts->total_rows)
-      return fail(ENGRAM_ERR_INVALID_ARG, "table %d (rows [%lld, %lld)) exceeds total_rows", h,
-                  static_cast<long long>(off), static_cast<long long>(off + wts->primes[h]));
-    hp.row_off[h] = off;
-  }
-  hp.ids = ids;
-  hp.lookup = wts->lookup;
-  hp.raw_vocab = wts->raw_vocab;
-  hp.history = history;
-  hp.status = dev_status;
-  hp.B = B;
-  hp.T = T;
+  if (static_cast<int64_t>(B) * T == 0) return ENGRAM_OK;
   HashGatherParams hg;
-  memset(&hg, 0, sizeof hg);
-  hg.h = hp;
-  hg.table = table;
-  hg.table_host = table_host ? 1 : 0;
-  hg.e = e;
-  hg.row_bytes = row_bytes;
+  st = prepare_gather(cfg, wts, ids, B, T, history, e, dev_status, &hg);
+  if (st != ENGRAM_OK) return st;
   return cuda_check(launch_hash_gather(hg, static_cast<cudaStream_t>(stream)), "hash+gather");
+}
+
+engram_status engram_gather_ids_layers(const engram_config* cfg, const engram_weights* const* layers,
+                                       int32_t n_layers, const int64_t* ids, int32_t B, int32_t T,
+                                       const int64_t* history, void* const* e, uint32_t* dev_status,
+                                       engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (n_layers < 1 || n_layers > ENGRAM_MAX_LAYERS)
+    return fail(ENGRAM_ERR_INVALID_ARG, "n_layers=%d outside [1, %d]", n_layers, ENGRAM_MAX_LAYERS);
+  if (layers == nullptr || e == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "layers / e arrays are NULL");
+  if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
+  if (static_cast<int64_t>(B) * T == 0) return ENGRAM_OK;
+  HashGatherLayers g;
+  memset(&g, 0, sizeof g);
+  g.n_layers = n_layers;
+  for (int l = 0; l < n_layers; ++l) {
+    st = prepare_gather(cfg, layers[l], ids, B, T, history, e[l], dev_status, &g.layer[l]);
+    if (st != ENGRAM_OK) return st;
+  }
+  return cuda_check(launch_hash_gather_layers(g, static_cast<cudaStream_t>(stream)), "hash+gather (layers)");
 }
 
 engram_status engram_forward_gathered(const engram_config* cfg, const engram_weights* wts, const void* e,

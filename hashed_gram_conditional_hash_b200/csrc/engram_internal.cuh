@@ -75,6 +75,12 @@ struct HashGatherParams {
   int32_t n_w;
 };
 cudaError_t launch_hash_gather(const HashGatherParams& p, cudaStream_t s);
+// Several layers' rows of the same ids in one launch (same shapes, row widths).
+struct HashGatherLayers {
+  HashGatherParams layer[ENGRAM_MAX_LAYERS];
+  int32_t n_layers;
+};
+cudaError_t launch_hash_gather_layers(const HashGatherLayers& p, cudaStream_t s);
 
 // Row gather (a4): e[m, h*Dh + c] = table[off[h] + idx[m, h], c].
 struct GatherParams {

@@ -138,8 +138,7 @@ __device__ __forceinline__ int4 ld_row_piece(const int4* p) {
 // Fewer rows per warp means more warps, each with one short dependent chain
 // (ids -> hash -> rows -> e), which is what the random row reads want.
 template <int CH, int ROWS, bool HOSTMEM>
-__global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant__ HashGatherParams g) {
-  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+__device__ __forceinline__ void hash_gather_body(const HashGatherParams& g) {
   const HashParams& p = g.h;
   const int lane = threadIdx.x & 31;
   const int gtid = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
@@ -194,6 +193,21 @@ __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant_
       if (i < per && q0 + r < total) out[i] = v[u];
     }
   }
+}
+
+template <int CH, int ROWS, bool HOSTMEM>
+__global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant__ HashGatherParams g) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  hash_gather_body<CH, ROWS, HOSTMEM>(g);
+}
+
+// Several Engram layers' rows of the same ids in one launch (blockIdx.y =
+// layer): the layers share the hashing structure and differ in multipliers,
+// primes, offsets and tables.
+template <int CH, int ROWS, bool HOSTMEM>
+__global__ void __launch_bounds__(256) hash_gather_layers_kernel(const __grid_constant__ HashGatherLayers g) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  hash_gather_body<CH, ROWS, HOSTMEM>(g.layer[blockIdx.y]);
 }
 
 __global__ void compress_kernel(const int64_t* __restrict__ raw, int64_t n,
@@ -251,6 +265,37 @@ cudaError_t launch_hash_gather(const HashGatherParams& g0, cudaStream_t s) {
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_hash_gather_layers(const HashGatherLayers& g0, cudaStream_t s) {
+  HashGatherLayers g = g0;
+  if (g.n_layers < 1 || g.n_layers > ENGRAM_MAX_LAYERS) return cudaErrorInvalidValue;
+  bool host = false;
+  for (int l = 0; l < g.n_layers; ++l) {
+    HashGatherParams& x = g.layer[l];
+    const HashParams& p = x.h;
+    x.div_nh = make_fastdiv(static_cast<uint32_t>(p.nh > 0 ? p.nh : 1));
+    x.div_J = make_fastdiv(static_cast<uint32_t>(p.J > 0 ? p.J : 1));
+    x.div_T = make_fastdiv(static_cast<uint32_t>(p.T > 0 ? p.T : 1));
+    host = host || x.table_host;
+    if (x.row_bytes != g.layer[0].row_bytes) return cudaErrorInvalidValue;
+  }
+  const HashParams& p = g.layer[0].h;
+  const int64_t total = static_cast<int64_t>(p.B) * p.T * p.nh;
+  if (total <= 0) return cudaSuccess;
+  constexpr int kRows = 16;
+  if (total * (32 / kRows) + 256 > INT32_MAX) return cudaErrorInvalidValue;
+  const unsigned layers = static_cast<unsigned>(g.n_layers);
+  if (g.layer[0].row_bytes == 128) {
+    const dim3 grid(static_cast<unsigned>((total + 8 * kRows - 1) / (8 * kRows)), layers);
+    if (host) launch_k(hash_gather_layers_kernel<8, kRows, true>, grid, dim3(256), 0, s, g);
+    else launch_k(hash_gather_layers_kernel<8, kRows, false>, grid, dim3(256), 0, s, g);
+  } else {
+    const dim3 grid(static_cast<unsigned>((total + 255) / 256), layers);
+    if (host) launch_k(hash_gather_layers_kernel<0, 32, true>, grid, dim3(256), 0, s, g);
+    else launch_k(hash_gather_layers_kernel<0, 32, false>, grid, dim3(256), 0, s, g);
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_compress(const int64_t* raw, int64_t n, const int64_t* lookup,

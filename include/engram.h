@@ -50,6 +50,7 @@ extern "C" {
 #define ENGRAM_MAX_HEADS 64   /* orders x heads per order */
 #define ENGRAM_MAX_HC 8       /* hyper-connection branches */
 #define ENGRAM_MAX_CONV_K 8   /* short-conv kernel length */
+#define ENGRAM_MAX_LAYERS 4   /* Engram layers gathered in one engram_gather_ids_layers call */
 
 typedef enum {
   ENGRAM_OK = 0,
@@ -278,6 +279,20 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wei
 engram_status engram_gather_ids(const engram_config* cfg, const engram_weights* weights, const int64_t* ids,
                                 int32_t B, int32_t T, const int64_t* history, void* e, uint32_t* dev_status,
                                 engram_stream stream);
+
+/* engram_gather_ids for several Engram layers of one model on the same ids,
+ * in one launch (the pages insert Engram at several layers, each with its own
+ * multipliers and tables, formulas §1.4; the hashes depend only on the ids,
+ * so all layers' rows can be fetched together ahead of the layers).
+ * layers[l]: the weights of layer l (table, total_rows, row_offsets, primes,
+ * multipliers, lookup, raw_vocab as in engram_gather_ids); e[l]: DEVICE
+ * [B*T, nh*Dh] output of layer l.  All layers share cfg (orders, heads, row
+ * width, dtype).  n_layers in [1, ENGRAM_MAX_LAYERS].  The rows of each layer
+ * are bit for bit those engram_gather_ids gives for it. */
+engram_status engram_gather_ids_layers(const engram_config* cfg, const engram_weights* const* layers,
+                                       int32_t n_layers, const int64_t* ids, int32_t B, int32_t T,
+                                       const int64_t* history, void* const* e, uint32_t* dev_status,
+                                       engram_stream stream);
 
 /* The rest of engram_forward (a5-a9) on rows gathered by engram_gather_ids:
  * y = the same result engram_forward gives for those ids (bit for bit on the

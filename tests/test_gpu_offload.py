@@ -91,3 +91,25 @@ def test_pageable_host_table_is_refused_without_launch():
     with pytest.raises(L.EngramError):
         layer.forward(p.ids, p.hidden)
     assert L.engram_launch_count() == before
+
+
+def test_gather_ids_layers_equals_per_layer_gathers():
+    # two Engram layers of one model (the pages' layers 2 and 6): own
+    # multipliers and tables, the same ids; one host-resident table
+    base = W.small_workload(B=3, T=90, orders=(2, 3, 4), heads_per_order=3)
+    ws_ = [base.replace(layer_id=2, seed=21), base.replace(layer_id=6, seed=22)]
+    ps = [device_params(w) for w in ws_]
+    ps[1].table = ps[1].table.cpu().pin_memory()
+    layers = [_layer(p) for p in ps]
+    ids = ps[0].ids
+    assert not np.array_equal(ps[0].mult, ps[1].mult)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    e = [torch.empty((base.B * base.T, base.nh * base.row_dim), dtype=ps[0].table.dtype, device=DEV)
+         for _ in layers]
+    L.engram_gather_ids_layers(layers[0].cfg, [l.weights for l in layers], ids, e, dev_status=st)
+    assert L.engram_read_status(st) == 0
+    for layer, e_l in zip(layers, e):
+        assert torch.equal(e_l, layer.gather_ids(ids))
+    # and the rows reach each layer's own forward
+    y0 = layers[0].forward_gathered(e[0], ps[0].hidden)
+    assert torch.equal(y0, layers[0].forward(ids, ps[0].hidden))
