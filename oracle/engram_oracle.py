@@ -11,7 +11,9 @@ arrays and composes the C steps:
 * ``forward``          - the whole pass over [B, T] with every input on the host;
 * ``forward_sampled``  - Y at chosen (b, t) positions only, for workloads whose
                          tables live on a device: the caller supplies a row
-                         fetcher, the oracle does the arithmetic.
+                         fetcher, the oracle does the arithmetic;
+* ``shard_table``, ``shard_route`` - the table split over R devices and the
+                         requests each device sends to the others (plain numpy).
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py
 (page worked example, closed forms, special cases and library cross-checks).
@@ -297,3 +299,28 @@ def forward_sampled(x, positions: Iterable[Tuple[int, int]], orders, J, mult, pr
         j = where[(b, t)]
         s_out[n], g_out[n] = s[j], g[j]
     return Y, s_out, g_out, idx
+
+
+# ---- a table sharded over R devices ---------------------------------------
+# The explainer page (§4.4, system efficiency) shards the tables across GPUs in
+# training and collects the active rows with an All-to-All; it fixes no split.
+# Reading used here: shard r of R holds the stacked table's rows r, r+R, r+2R,
+# ... (row -> shard row % R, local row row // R), so that every head's rows
+# and every skewed id spread evenly over the shards.
+
+def shard_table(table: np.ndarray, n_shards: int, r: int) -> np.ndarray:
+    """Shard r of n_shards: rows r, r + n_shards, ... of the stacked table."""
+    return np.ascontiguousarray(table[r::n_shards])
+
+
+def shard_route(rows, n_shards: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Requests of the sharded gather of absolute rows ``rows`` (one per row q
+    of e, q = m*nh + h, in that order).  Returns (counts [R], req_rows [N],
+    req_pos [N]): the requests grouped by shard (shard 0 first), in increasing
+    q within a shard; request k asks its shard for local row req_rows[k] and
+    fills row req_pos[k] of e; counts[r] requests go to shard r."""
+    rows = _i64(rows).reshape(-1)
+    owner = rows % n_shards
+    order = np.argsort(owner, kind="stable")      # group by shard, q order kept
+    counts = np.bincount(owner, minlength=n_shards).astype(np.int64)
+    return counts, (rows // n_shards)[order], order.astype(np.int32)

@@ -175,6 +175,44 @@ def test_compress_and_gather_match_numpy_take():
     assert e.dtype == np.uint16
 
 
+# ---------------------------------------------------------------- sharded table
+
+def test_shard_route_hand_example():
+    # rows 5 2 7 4 0 3 over 3 shards: owners 2 2 1 1 0 0, local rows 1 0 2 1 0 1
+    counts, req_rows, req_pos = O.shard_route(np.array([5, 2, 7, 4, 0, 3]), 3)
+    assert counts.tolist() == [2, 2, 2]
+    assert req_pos.tolist() == [4, 5, 2, 3, 0, 1]
+    assert req_rows.tolist() == [0, 1, 2, 1, 1, 0]
+
+
+def test_shard_route_brute_force_and_reassembly():
+    rng = np.random.default_rng(5)
+    table = rng.integers(0, 1 << 16, size=(97, 8)).astype(np.uint16)
+    rows = rng.integers(0, 97, size=300)
+    for R in (1, 2, 3, 8):
+        counts, req_rows, req_pos = O.shard_route(rows, R)
+        # brute force: walk q in order, append to its shard's list
+        lists = [[] for _ in range(R)]
+        for q, row in enumerate(rows.tolist()):
+            lists[row % R].append((row // R, q))
+        flat = [x for lst in lists for x in lst]
+        assert counts.tolist() == [len(l) for l in lists]
+        assert req_rows.tolist() == [a for a, _ in flat]
+        assert req_pos.tolist() == [b for _, b in flat]
+        # serving each shard's requests from its shard and placing them at
+        # req_pos gives the plain gather of the full table
+        shards = [O.shard_table(table, R, r) for r in range(R)]
+        assert sum(len(sh) for sh in shards) == len(table)
+        owner = np.repeat(np.arange(R), counts)
+        got = np.stack([shards[o][k] for o, k in zip(owner, req_rows)])
+        e = np.empty_like(table[rows])
+        e[req_pos] = got
+        np.testing.assert_array_equal(e, table[rows])
+    c1, r1, p1 = O.shard_route(rows, 1)
+    np.testing.assert_array_equal(r1, rows)
+    np.testing.assert_array_equal(p1, np.arange(len(rows)))
+
+
 def test_widen_bf16_is_exact():
     t = torch.randn(1000, dtype=torch.float32).to(torch.bfloat16)
     a, code = O.storage(t)
