@@ -381,6 +381,7 @@ constexpr int kTileTMin = 32;     // positions per block: the launcher picks one
 constexpr int kTileTMax = 64;     // [32, 64] that spreads the blocks evenly over the SMs
 constexpr int kTileC = 256;       // channels per block (512 bytes of a bf16 row)
 constexpr int kTileMaxDil = 32;   // longer halos take the run form
+constexpr int kStepSeq = 4;       // sequences per block of the decode step
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -549,51 +550,45 @@ __global__ void __launch_bounds__((kTileC / CPL) * ENGRAM_MAX_HC) conv_tile_kern
   }
 }
 
-// One decode step (T = 1) with the streaming state, K = 4 taps, bfloat16,
-// 256-channel slices: block (sequence b, slice), one warp per branch, 8
-// channels per lane.  Every lane loads its 16-byte piece of V(t) and the
-// step's gate, turns pos into the ring rows of the taps at t - 3 dil,
-// t - 2 dil, t - dil itself (the ring holds (K-1) dil + 1 >= 3 dil + 1
+// One decode step (T = 1) with the streaming state, K = 4 taps, bfloat16:
+// block (group of kStepSeq sequences, 256-channel slice), one warp per
+// branch, 8 channels per lane.  A lane loads its taps once for the group,
+// then, for every sequence of the group at once, its 16-byte piece of V(t),
+// the step's gate and pos; turns pos into the ring rows of the taps at
+// t - 3 dil, t - 2 dil, t - dil (the ring holds (K-1) dil + 1 >= 3 dil + 1
 // positions, slot = position mod ring length, by invariant-divisor
-// multiplication), loads its pieces of those three rows, their gates and its
-// taps, and stores 8 channels of Y; no block barrier.  The same kernel is the
+// multiplication) and loads its pieces of those rows and their gates, so that
+// each lane has every sequence's loads in flight together; then it stores 8
+// channels of Y per sequence.  No block barrier.  The same kernel is the
 // step's state advance: the branch-0 warp writes V(t) and lanes 0 write g(t)
 // into t's slot, which no tap of this step reads.
+template <int S>
 __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __grid_constant__ ConvParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   constexpr int K = 4;
-  const int b = static_cast<int>(blockIdx.x);
   const int tid = static_cast<int>(threadIdx.x);
   const int h = tid >> 5, lane = tid & 31;
   if (h >= p.hc) return;
+  const int b0 = static_cast<int>(blockIdx.x) * S;
   const int c = static_cast<int>(blockIdx.y) * kTileC + lane * 8;
   const uint16_t* V = static_cast<const uint16_t*>(p.V);
   uint16_t* vr = static_cast<uint16_t*>(const_cast<void*>(p.v_ring));
   float* gr = const_cast<float*>(p.g_ring);
-  uint4 raw[K];
-  float gg[K];
-  // what does not depend on the ring first, then every thread turns pos into
-  // the ring rows of its taps itself (no block barrier on the way)
-  raw[K - 1] = __ldg(reinterpret_cast<const uint4*>(V + static_cast<int64_t>(b) * p.H + c));
-  gg[K - 1] = __ldg(p.g + static_cast<int64_t>(b) * p.hc + h);
-  const int64_t P = __ldg(p.pos + b) - p.pos_lag;   // position of this step's token
-  const int64_t slot_t = (P >= 0 && P < INT32_MAX)
-                             ? static_cast<int64_t>(P - static_cast<int64_t>(fast_div(static_cast<uint32_t>(P), p.div_ring)) *
-                                                            p.ring_len)
-                             : P % p.ring_len;
-  const int64_t ring0 = static_cast<int64_t>(b) * p.ring_len;
+  uint4 raw[S][K];
+  float gg[S][K];
+  int64_t P[S];
+  // what does not depend on the ring, for the whole group
 #pragma unroll
-  for (int i = 0; i < K - 1; ++i) {                 // tap i sits at t - (K-1-i) dil
-    const int64_t back = static_cast<int64_t>(K - 1 - i) * p.dil;
-    int64_t slot = slot_t - back;
-    if (slot < 0) slot += p.ring_len;
-    if (P - back >= 0) {
-      const int64_t row = ring0 + slot;
-      raw[i] = __ldg(reinterpret_cast<const uint4*>(vr + row * p.H + c));
-      gg[i] = __ldg(gr + row * p.hc + h);
+  for (int s = 0; s < S; ++s) {
+    const int b = b0 + s;
+    if (b < p.B) {
+      raw[s][K - 1] = __ldg(reinterpret_cast<const uint4*>(V + static_cast<int64_t>(b) * p.H + c));
+      gg[s][K - 1] = __ldg(p.g + static_cast<int64_t>(b) * p.hc + h);
+      P[s] = __ldg(p.pos + b) - p.pos_lag;          // position of this step's token
     } else {
-      raw[i] = make_uint4(0, 0, 0, 0);
-      gg[i] = 0.f;
+      raw[s][K - 1] = make_uint4(0, 0, 0, 0);
+      gg[s][K - 1] = 0.f;
+      P[s] = -1;
     }
   }
   float2 w2[4][K];                                // [channel pair][tap]
@@ -605,28 +600,58 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __g
 #pragma unroll
       for (int i = 0; i < K; ++i) w2[j][i] = make_float2(w[2 * j][i], w[2 * j + 1][i]);
   }
-  float2 u[K][4];
+  // the ring rows of the taps, for the whole group
+  int64_t row_t[S];
 #pragma unroll
-  for (int i = 0; i < K; ++i) {
-    float2 v[4];
-    Pair8<uint16_t>::unpack(raw[i], v);
-    const float2 g2 = make_float2(gg[i], gg[i]);
+  for (int s = 0; s < S; ++s) {
+    const int64_t Ps = P[s];
+    const int64_t slot_t = (Ps >= 0 && Ps < INT32_MAX)
+                               ? static_cast<int64_t>(Ps - static_cast<int64_t>(fast_div(static_cast<uint32_t>(Ps), p.div_ring)) *
+                                                              p.ring_len)
+                               : (Ps >= 0 ? Ps % p.ring_len : 0);
+    const int64_t ring0 = static_cast<int64_t>(b0 + s) * p.ring_len;
+    row_t[s] = ring0 + slot_t;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) u[i][j] = __fmul2_rn(g2, v[j]);
+    for (int i = 0; i < K - 1; ++i) {               // tap i sits at t - (K-1-i) dil
+      const int64_t back = static_cast<int64_t>(K - 1 - i) * p.dil;
+      int64_t slot = slot_t - back;
+      if (slot < 0) slot += p.ring_len;
+      if (Ps - back >= 0) {                         // also false past the last sequence (P = -1)
+        const int64_t row = ring0 + slot;
+        raw[s][i] = __ldg(reinterpret_cast<const uint4*>(vr + row * p.H + c));
+        gg[s][i] = __ldg(gr + row * p.hc + h);
+      } else {
+        raw[s][i] = make_uint4(0, 0, 0, 0);
+        gg[s][i] = 0.f;
+      }
+    }
   }
-  float2 acc[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    float2 a = u[K - 1][j];
+  for (int s = 0; s < S; ++s) {
+    const int b = b0 + s;
+    if (b >= p.B) break;
+    float2 u[K][4];
 #pragma unroll
-    for (int i = 0; i < K; ++i) a = __ffma2_rn(w2[j][i], u[i][j], a);
-    acc[j] = a;
+    for (int i = 0; i < K; ++i) {
+      float2 v[4];
+      Pair8<uint16_t>::unpack(raw[s][i], v);
+      const float2 g2 = make_float2(gg[s][i], gg[s][i]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) u[i][j] = __fmul2_rn(g2, v[j]);
+    }
+    float2 acc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 a = u[K - 1][j];
+#pragma unroll
+      for (int i = 0; i < K; ++i) a = __ffma2_rn(w2[j][i], u[i][j], a);
+      acc[j] = a;
+    }
+    Pair8<uint16_t>::store(static_cast<uint16_t*>(p.Y) + (static_cast<int64_t>(b) * p.hc + h) * p.H + c, acc);
+    // the step's state advance
+    if (h == 0) *reinterpret_cast<uint4*>(vr + row_t[s] * p.H + c) = raw[s][K - 1];
+    if (blockIdx.y == 0 && lane == 0) gr[row_t[s] * p.hc + h] = gg[s][K - 1];
   }
-  Pair8<uint16_t>::store(static_cast<uint16_t*>(p.Y) + (static_cast<int64_t>(b) * p.hc + h) * p.H + c, acc);
-  // the step's state advance
-  const int64_t row_t = ring0 + slot_t;
-  if (h == 0) *reinterpret_cast<uint4*>(vr + row_t * p.H + c) = raw[K - 1];
-  if (blockIdx.y == 0 && lane == 0) gr[row_t * p.hc + h] = gg[K - 1];
 }
 
 // -------------------------------------------------------------- standalone conv
@@ -744,7 +769,8 @@ cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {
   if (conv_writes_rings(p)) {
     ConvParams q = p;
     q.div_ring = make_fastdiv(static_cast<uint32_t>(p.ring_len));
-    launch_k(conv_step_kernel, dim3(static_cast<unsigned>(p.B), static_cast<unsigned>(p.H / kTileC)),
+    launch_k(conv_step_kernel<kStepSeq>,
+             dim3(static_cast<unsigned>((p.B + kStepSeq - 1) / kStepSeq), static_cast<unsigned>(p.H / kTileC)),
              dim3(32 * p.hc), 0, s, q);
     return cudaGetLastError();
   }
