@@ -526,6 +526,73 @@ def run_offload(args, layer, p, w, device):
                     "layers' compute to hide the host-link transfer behind"}
 
 
+PEER_COPY_GBS = 770.0   # NVLink 5 peer copy rate measured on B200 HGX, per direction per GPU
+
+
+def run_sharded(args, layer, p, w, device):
+    """The table sharded over R GPUs (explainer §4.4), on ONE GPU: the device
+    steps of one rank's gather timed against the plain hash + gather of the
+    same ids (L2 flushed between steps).  route = engram_shard_route (3
+    kernels); serve = the rows one rank serves per step: every rank asks about
+    N/R rows of each shard, so a rank serves about N rows of its shard in one
+    launch (timed as the N local rows of this batch served from shard 0, the
+    largest, of total/R rows); place = engram_shard_place.  The two
+    all-to-alls cannot run on one GPU: their per-rank bytes are reported with
+    the time they would take at the measured peer-copy rate, as an estimate."""
+    from hashed_gram_conditional_hash_b200 import _lib as L
+    R = args.sharded
+    B, T = w.B, w.T
+    n = B * T * w.nh
+    rb = w.row_dim * p.table.element_size()
+    counts = torch.empty(R, dtype=torch.int64, device=device)
+    req_rows = torch.empty(n, dtype=torch.int64, device=device)
+    req_pos = torch.empty(n, dtype=torch.int32, device=device)
+    ws = torch.empty(max(L.engram_shard_route_workspace_size(layer.cfg, B, T, R), 256), dtype=torch.uint8,
+                     device=device)
+    shard0 = p.table[0::R].contiguous()
+    got = torch.empty((n, w.row_dim), dtype=p.table.dtype, device=device)
+    e = torch.empty((B * T, w.nh * w.row_dim), dtype=p.table.dtype, device=device)
+    L.engram_shard_route(layer.cfg, layer.weights, p.ids, R, counts, req_rows, req_pos, ws)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    K = max(3, min(args.steps, 200))
+
+    def timed(step):
+        for i in range(3):
+            step()
+            flush.fill_(i & 0xff)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(K):
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+            flush.fill_(i & 0xff)
+        torch.cuda.synchronize()
+        return sorted(a.elapsed_time(b) * 1e3 for a, b in ev)[K // 2]     # median µs
+
+    t_plain = timed(lambda: layer.gather_ids(p.ids, e=e))
+    t_route = timed(lambda: L.engram_shard_route(layer.cfg, layer.weights, p.ids, R, counts, req_rows, req_pos, ws))
+    t_serve = timed(lambda: L.engram_shard_serve(layer.cfg, shard0, req_rows, got))
+    t_place = timed(lambda: L.engram_shard_place(layer.cfg, got, req_pos, e, n))
+
+    def steps():
+        L.engram_shard_route(layer.cfg, layer.weights, p.ids, R, counts, req_rows, req_pos, ws)
+        L.engram_shard_serve(layer.cfg, shard0, req_rows, got)
+        L.engram_shard_place(layer.cfg, got, req_pos, e, n)
+    t_steps = timed(steps)
+    remote = n * (R - 1) / R                       # requests of one rank that leave the GPU
+    x_bytes = remote * (8 + rb)                    # local row ids out + rows back, per direction
+    return {"shards": R, "requests_per_rank": n, "row_bytes": rb,
+            "plain_hash_gather_us": t_plain, "route_us": t_route, "serve_us": t_serve, "place_us": t_place,
+            "device_steps_us": t_steps,
+            "exchange_bytes_per_rank_each_way": int(x_bytes),
+            "exchange_us_estimated": x_bytes / (PEER_COPY_GBS * 1e3),
+            "note": "one GPU: device steps measured (medians, L2 flushed before each timed launch, so each "
+                    "part alone also pays the flush's write-back; device_steps_us is the three back to back "
+                    "after one flush); the two all-to-alls estimated from their bytes at %.0f GB/s per "
+                    "direction, not measured" % PEER_COPY_GBS}
+
+
 def run_reference(args):
     """The reference arm: the float64 oracle on the host cores, K timed steps
     of a bounded sample each, sized so that warm-up + steps take ~2 minutes."""
@@ -570,6 +637,8 @@ def main():
                     help="decode workload: number of distinct calls drawn (default: all 256)")
     ap.add_argument("--offload", action="store_true",
                     help="also measure tables resident in pinned host memory (prefill workloads)")
+    ap.add_argument("--sharded", type=int, default=0,
+                    help="also time the device steps of a gather from a table sharded over this many GPUs")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -593,6 +662,8 @@ def main():
             res["e2e"] = run_e2e(args, layer, p, w, device, world)
         if args.offload and not w.decode_calls:
             res["offload"] = run_offload(args, layer, p, w, device)
+        if args.sharded and not w.decode_calls:
+            res["sharded"] = run_sharded(args, layer, p, w, device)
         del layer, p
         torch.cuda.empty_cache()
         if rank == 0 and not args.no_cpu_baseline and world == 1:

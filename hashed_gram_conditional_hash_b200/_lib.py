@@ -98,6 +98,12 @@ def lib() -> C.CDLL:
             "engram_gather_ids": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P, P, P, P]),
             "engram_forward_gathered": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P, P, P, sz,
                                                   P, P]),
+            "engram_shard_rows": (i64, [i64, i32, i32]),
+            "engram_shard_route_workspace_size": (sz, [cfg, i32, i32, i32]),
+            "engram_shard_route": (C.c_int, [cfg, C.POINTER(EngramWeights), P, i32, i32, P, i32, P, P, P, P, sz,
+                                             P, P]),
+            "engram_shard_serve": (C.c_int, [cfg, P, i64, P, i64, P, P, P]),
+            "engram_shard_place": (C.c_int, [cfg, P, P, i64, P, i64, P, P]),
             "engram_gather_ids_layers": (C.c_int, [cfg, C.POINTER(C.POINTER(EngramWeights)), i32, P, i32, i32,
                                                    P, C.POINTER(P), P, P]),
         }
@@ -304,6 +310,43 @@ def engram_gather_ids_layers(cfg: EngramConfig, weights: Sequence[EngramWeights]
     ep = (C.c_void_p * n)(*[_ptr(t).value for t in e])
     _check(lib().engram_gather_ids_layers(C.byref(cfg), wp, n, _ptr(ids), B, T, _ptr(history), ep,
                                           _ptr(dev_status), _stream(stream)))
+
+
+MAX_SHARDS = 64
+
+
+def engram_shard_rows(total_rows: int, n_shards: int, shard: int) -> int:
+    """Rows held by shard ``shard`` (stacked-table rows shard, shard + n_shards, ...)."""
+    n = lib().engram_shard_rows(total_rows, n_shards, shard)
+    if n < 0:
+        raise ValueError("shard %d of %d out of range" % (shard, n_shards))
+    return n
+
+
+def engram_shard_route_workspace_size(cfg: EngramConfig, B: int, T: int, n_shards: int) -> int:
+    return lib().engram_shard_route_workspace_size(C.byref(cfg), B, T, n_shards)
+
+
+def engram_shard_route(cfg: EngramConfig, weights: EngramWeights, ids: torch.Tensor, n_shards: int,
+                       counts: torch.Tensor, req_rows: torch.Tensor, req_pos: torch.Tensor, ws: torch.Tensor,
+                       history: Optional[torch.Tensor] = None, dev_status: Optional[torch.Tensor] = None,
+                       stream=None) -> None:
+    B, T = ids.shape
+    _check(lib().engram_shard_route(C.byref(cfg), C.byref(weights), _ptr(ids), B, T, _ptr(history), n_shards,
+                                    _ptr(counts), _ptr(req_rows), _ptr(req_pos), _ptr(ws), ws.numel(),
+                                    _ptr(dev_status), _stream(stream)))
+
+
+def engram_shard_serve(cfg: EngramConfig, shard: torch.Tensor, req_rows: torch.Tensor, out: torch.Tensor,
+                       dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(lib().engram_shard_serve(C.byref(cfg), _ptr(shard), shard.shape[0], _ptr(req_rows), req_rows.numel(),
+                                    _ptr(out), _ptr(dev_status), _stream(stream)))
+
+
+def engram_shard_place(cfg: EngramConfig, got: torch.Tensor, req_pos: torch.Tensor, e: torch.Tensor,
+                       n_e: int, dev_status: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(lib().engram_shard_place(C.byref(cfg), _ptr(got), _ptr(req_pos), req_pos.numel(), _ptr(e), n_e,
+                                    _ptr(dev_status), _stream(stream)))
 
 
 def engram_forward_gathered(cfg: EngramConfig, weights: EngramWeights, e: torch.Tensor, B: int, T: int,

@@ -214,25 +214,32 @@ engram_status run_stage(const engram_config* c, ProjParams pp, float* g, float* 
 }
 
 // Checks and fills the parameters of the hash + gather of one layer's rows
-// into e (engram_gather_ids and engram_gather_ids_layers); B*T > 0.
+// into e (engram_gather_ids, engram_gather_ids_layers; with_table false: the
+// hash alone, for engram_shard_route, which reads neither table nor e);
+// B*T > 0.
 engram_status prepare_gather(const engram_config* cfg, const engram_weights* wts, const int64_t* ids,
                              int32_t B, int32_t T, const int64_t* history, void* e, uint32_t* dev_status,
-                             HashGatherParams* hg) {
+                             HashGatherParams* hg, bool with_table = true) {
   if (wts == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights is NULL");
   const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
   if (row_bytes % 16 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
-  if (wts->table == nullptr || ids == nullptr || e == nullptr)
-    return fail(ENGRAM_ERR_INVALID_ARG, "table / ids / e must be non-NULL");
-  if (!aligned16(e) || !aligned16(ids)) return fail(ENGRAM_ERR_INVALID_ARG, "ids and e must be 16-byte aligned");
+  if (ids == nullptr || !aligned16(ids)) return fail(ENGRAM_ERR_INVALID_ARG, "ids must be non-NULL, 16-byte aligned");
+  if (with_table) {
+    if (wts->table == nullptr || e == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "table / e must be non-NULL");
+    if (!aligned16(e)) return fail(ENGRAM_ERR_INVALID_ARG, "e must be 16-byte aligned");
+  }
   if (wts->row_offsets == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "row_offsets (host) is NULL");
   if (wts->lookup != nullptr && wts->raw_vocab < 1) return fail(ENGRAM_ERR_INVALID_ARG, "raw_vocab < 1");
   if (wts->total_rows < 1 || wts->total_rows > INT32_MAX)
     return fail(ENGRAM_ERR_UNSUPPORTED, "total_rows must be in [1, 2^31)");
   const void* table = nullptr;
   bool table_host = false;
-  engram_status st = table_location(wts->table, &table, &table_host);
-  if (st != ENGRAM_OK) return st;
-  if (!aligned16(table)) return fail(ENGRAM_ERR_INVALID_ARG, "table must be 16-byte aligned");
+  engram_status st = ENGRAM_OK;
+  if (with_table) {
+    st = table_location(wts->table, &table, &table_host);
+    if (st != ENGRAM_OK) return st;
+    if (!aligned16(table)) return fail(ENGRAM_ERR_INVALID_ARG, "table must be 16-byte aligned");
+  }
   HashParams hp;
   st = fill_hash_params(cfg, wts->multipliers, wts->primes, &hp);
   if (st != ENGRAM_OK) return st;
@@ -771,6 +778,108 @@ engram_status engram_forward_gathered(const engram_config* cfg, const engram_wei
   const int nh = cfg->n_orders * cfg->heads_per_order;
   return forward_tail(cfg, wts, L, static_cast<char*>(ws), e, nullptr, rows_ld(M), nullptr, nh, 0, nullptr, B, T,
                       hidden, y, nullptr, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+// ---- a table sharded over several devices
+
+int64_t engram_shard_rows(int64_t total_rows, int32_t n_shards, int32_t shard) {
+  if (total_rows < 0 || n_shards < 1 || shard < 0 || shard >= n_shards) return -1;
+  return total_rows > shard ? (total_rows - shard + n_shards - 1) / n_shards : 0;
+}
+
+size_t engram_shard_route_workspace_size(const engram_config* cfg, int32_t B, int32_t T, int32_t n_shards) {
+  if (cfg == nullptr || B < 0 || T < 0 || n_shards < 1) return 0;
+  const int64_t n = static_cast<int64_t>(B) * T * cfg->n_orders * cfg->heads_per_order;
+  const int64_t blk = (n + kShardChunk - 1) / kShardChunk;
+  return align256(static_cast<size_t>(n) * sizeof(int64_t)) +
+         align256(static_cast<size_t>(blk) * n_shards * sizeof(int32_t));
+}
+
+engram_status engram_shard_route(const engram_config* cfg, const engram_weights* wts, const int64_t* ids,
+                                 int32_t B, int32_t T, const int64_t* history, int32_t n_shards, int64_t* counts,
+                                 int64_t* req_rows, int32_t* req_pos, void* ws, size_t ws_bytes,
+                                 uint32_t* dev_status, engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
+  if (n_shards < 1 || n_shards > ENGRAM_MAX_SHARDS)
+    return fail(ENGRAM_ERR_INVALID_ARG, "n_shards=%d outside [1, %d]", n_shards, ENGRAM_MAX_SHARDS);
+  if (counts == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "counts is NULL");
+  const int64_t n = static_cast<int64_t>(B) * T * cfg->n_orders * cfg->heads_per_order;
+  if (n + kShardChunk > INT32_MAX) return fail(ENGRAM_ERR_UNSUPPORTED, "B*T*nh must stay below 2^31");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (n == 0)
+    return cuda_check(cudaMemsetAsync(counts, 0, sizeof(int64_t) * n_shards, s), "route counts");
+  if (req_rows == nullptr || req_pos == nullptr || ws == nullptr)
+    return fail(ENGRAM_ERR_INVALID_ARG, "req_rows / req_pos / ws must be non-NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(ENGRAM_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+  const size_t need = engram_shard_route_workspace_size(cfg, B, T, n_shards);
+  if (ws_bytes < need) return fail(ENGRAM_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  ShardRouteParams p;
+  memset(&p, 0, sizeof p);
+  st = prepare_gather(cfg, wts, ids, B, T, history, nullptr, dev_status, &p.g, false);
+  if (st != ENGRAM_OK) return st;
+  p.n_shards = n_shards;
+  p.rows = static_cast<int64_t*>(ws);
+  p.blk_cnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align256(static_cast<size_t>(n) * sizeof(int64_t)));
+  p.counts = counts;
+  p.req_rows = req_rows;
+  p.req_pos = req_pos;
+  return cuda_check(launch_shard_route(p, s), "shard route");
+}
+
+engram_status engram_shard_serve(const engram_config* cfg, const void* shard, int64_t shard_rows,
+                                 const int64_t* req_rows, int64_t n, void* out, uint32_t* dev_status,
+                                 engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (n < 0 || shard_rows < 0) return fail(ENGRAM_ERR_INVALID_ARG, "n, shard_rows must be >= 0");
+  if (n == 0) return ENGRAM_OK;
+  const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
+  if (row_bytes % 16 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
+  if (shard == nullptr || req_rows == nullptr || out == nullptr)
+    return fail(ENGRAM_ERR_INVALID_ARG, "shard / req_rows / out must be non-NULL");
+  if (!aligned16(shard) || !aligned16(out)) return fail(ENGRAM_ERR_INVALID_ARG, "shard and out must be 16-byte aligned");
+  const void* dev = nullptr;
+  bool host = false;
+  st = table_location(shard, &dev, &host);
+  if (st != ENGRAM_OK) return st;
+  if (host) return fail(ENGRAM_ERR_INVALID_ARG, "the shard must be device memory");
+  GatherParams g;
+  memset(&g, 0, sizeof g);
+  g.table = shard;
+  g.idx = req_rows;
+  g.e = out;
+  g.status = dev_status;
+  g.M = n;
+  g.total_rows = shard_rows;
+  g.nh = 1;
+  g.row_bytes = row_bytes;
+  g.row_off[0] = 0;
+  return cuda_check(launch_gather(g, static_cast<cudaStream_t>(stream)), "shard serve");
+}
+
+engram_status engram_shard_place(const engram_config* cfg, const void* got, const int32_t* req_pos, int64_t n,
+                                 void* e, int64_t n_e, uint32_t* dev_status, engram_stream stream) {
+  engram_status st = check_config(cfg);
+  if (st != ENGRAM_OK) return st;
+  if (n < 0 || n_e < 0) return fail(ENGRAM_ERR_INVALID_ARG, "n, n_e must be >= 0");
+  if (n == 0) return ENGRAM_OK;
+  const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
+  if (row_bytes % 16 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
+  if (got == nullptr || req_pos == nullptr || e == nullptr)
+    return fail(ENGRAM_ERR_INVALID_ARG, "got / req_pos / e must be non-NULL");
+  if (!aligned16(got) || !aligned16(e)) return fail(ENGRAM_ERR_INVALID_ARG, "got and e must be 16-byte aligned");
+  PlaceParams p;
+  p.got = got;
+  p.pos = req_pos;
+  p.e = e;
+  p.status = dev_status;
+  p.n = n;
+  p.n_out = n_e;
+  p.row_bytes = row_bytes;
+  return cuda_check(launch_place(p, static_cast<cudaStream_t>(stream)), "shard place");
 }
 
 }  // extern "C"

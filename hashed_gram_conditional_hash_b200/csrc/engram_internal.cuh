@@ -82,6 +82,36 @@ struct HashGatherLayers {
 };
 cudaError_t launch_hash_gather_layers(const HashGatherLayers& p, cudaStream_t s);
 
+// A table sharded over R devices: shard r holds the stacked table's rows
+// r, r+R, r+2R, ... (row -> shard row mod R, local row row / R).  The route
+// hashes every row q = m*nh + h of e and lists the requests grouped by shard,
+// in increasing q within a shard (a stable counting sort over blocks of
+// kShardChunk requests: per-block counts, a per-shard scan over the blocks,
+// then a stable scatter).
+constexpr int kShardChunk = 256;
+struct ShardRouteParams {
+  HashGatherParams g;       // the layer's hash (table and e unused)
+  int32_t n_shards;
+  FastDiv div_shards;
+  int32_t n_blk;            // ceil(N / kShardChunk), N = B*T*nh
+  int64_t* rows;            // [N] scratch: absolute row of each request
+  int32_t* blk_cnt;         // [n_blk, n_shards] scratch: counts, then offsets
+  int64_t* counts;          // [n_shards] out
+  int64_t* req_rows;        // [N] out: local row inside the shard
+  int32_t* req_pos;         // [N] out: the row q of e the request fills
+};
+cudaError_t launch_shard_route(const ShardRouteParams& p, cudaStream_t s);
+// e[pos[k]] = got[k] for the rows a sharded gather received (row_bytes % 16 == 0).
+struct PlaceParams {
+  const void* got;          // [n, row_bytes]
+  const int32_t* pos;       // [n]
+  void* e;                  // [n_out, row_bytes]
+  uint32_t* status;
+  int64_t n, n_out;
+  int32_t row_bytes;
+};
+cudaError_t launch_place(const PlaceParams& p, cudaStream_t s);
+
 // Row gather (a4): e[m, h*Dh + c] = table[off[h] + idx[m, h], c].
 struct GatherParams {
   const void* table;

@@ -210,6 +210,119 @@ __global__ void __launch_bounds__(256) hash_gather_layers_kernel(const __grid_co
   hash_gather_body<CH, ROWS, HOSTMEM>(g.layer[blockIdx.y]);
 }
 
+// ---- routing of a sharded gather
+// Block x of the route owns requests [x*kShardChunk, (x+1)*kShardChunk).
+
+__device__ __forceinline__ int shard_of(int64_t row, const ShardRouteParams& p, uint32_t* local) {
+  const uint32_t r32 = static_cast<uint32_t>(row);   // row < total_rows < 2^31
+  const uint32_t l = fast_div(r32, p.div_shards);
+  *local = l;
+  return static_cast<int>(r32 - l * static_cast<uint32_t>(p.n_shards));
+}
+
+// Pass 1: hash every request of the block, keep its row, count per shard.
+__global__ void __launch_bounds__(kShardChunk) shard_count_kernel(const __grid_constant__ ShardRouteParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  __shared__ int cnt[ENGRAM_MAX_SHARDS];
+  const int tid = static_cast<int>(threadIdx.x);
+  for (int r = tid; r < p.n_shards; r += kShardChunk) cnt[r] = 0;
+  __syncthreads();
+  const int total = p.g.h.B * p.g.h.T * p.g.h.nh;
+  const int q = static_cast<int>(blockIdx.x) * kShardChunk + tid;
+  if (q < total) {
+    const int64_t row = hashed_row(p.g, q);
+    p.rows[q] = row;
+    uint32_t local;
+    atomicAdd(&cnt[shard_of(row, p, &local)], 1);
+  }
+  __syncthreads();
+  for (int r = tid; r < p.n_shards; r += kShardChunk)
+    p.blk_cnt[static_cast<int64_t>(blockIdx.x) * p.n_shards + r] = cnt[r];
+}
+
+// Pass 2 (block r = shard r): exclusive scan of shard r's per-block counts
+// over the blocks, in place; counts[r] = the shard's total.
+__global__ void __launch_bounds__(1024) shard_scan_kernel(const __grid_constant__ ShardRouteParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  __shared__ int wsum[32];
+  const int r = static_cast<int>(blockIdx.x);
+  const int tid = static_cast<int>(threadIdx.x), lane = tid & 31, w = tid >> 5;
+  const int per = (p.n_blk + 1023) / 1024;
+  const int b0 = min(tid * per, p.n_blk), b1 = min(b0 + per, p.n_blk);
+  int own = 0;
+  for (int b = b0; b < b1; ++b) own += p.blk_cnt[static_cast<int64_t>(b) * p.n_shards + r];
+  int x = own;                                       // inclusive scan in the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[w] = x;
+  __syncthreads();
+  if (w == 0) {                                      // scan of the 32 warp sums
+    int v = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    wsum[lane] = v;
+  }
+  __syncthreads();
+  int run = x - own + (w > 0 ? wsum[w - 1] : 0);     // requests of shard r before block b0
+  for (int b = b0; b < b1; ++b) {
+    int* c = p.blk_cnt + static_cast<int64_t>(b) * p.n_shards + r;
+    const int n = *c;
+    *c = run;
+    run += n;
+  }
+  if (tid == 0) p.counts[r] = wsum[31];
+}
+
+// Pass 3: every request to its place.  Within a warp, lanes asking the same
+// shard rank themselves by lane (match_any); warps of the block stack in
+// order; blocks stack by the scanned offsets; shards by their counts.  The
+// result is the stable grouping: increasing q within a shard.
+__global__ void __launch_bounds__(kShardChunk) shard_scatter_kernel(const __grid_constant__ ShardRouteParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  constexpr int kWarps = kShardChunk / 32;
+  __shared__ int first[ENGRAM_MAX_SHARDS];           // first slot of shard r for this block
+  __shared__ int wcnt[kWarps][ENGRAM_MAX_SHARDS];    // per-warp counts, then offsets
+  const int tid = static_cast<int>(threadIdx.x), lane = tid & 31, w = tid >> 5;
+  const int R = p.n_shards;
+  for (int i = tid; i < kWarps * ENGRAM_MAX_SHARDS; i += kShardChunk) (&wcnt[0][0])[i] = 0;
+  if (tid < R) {
+    int64_t before = 0;
+    for (int r = 0; r < tid; ++r) before += p.counts[r];
+    first[tid] = static_cast<int>(before) + p.blk_cnt[static_cast<int64_t>(blockIdx.x) * R + tid];
+  }
+  __syncthreads();
+  const int total = p.g.h.B * p.g.h.T * p.g.h.nh;
+  const int q = static_cast<int>(blockIdx.x) * kShardChunk + tid;
+  const bool live = q < total;
+  uint32_t local = 0;
+  const int own = live ? shard_of(p.rows[q], p, &local) : -1;
+  const unsigned peers = __match_any_sync(0xffffffffu, own);
+  const int rank = __popc(peers & ((1u << lane) - 1u));
+  if (live && rank == 0) wcnt[w][own] = __popc(peers);
+  __syncthreads();
+  if (tid < R) {
+    int run = 0;
+#pragma unroll
+    for (int k = 0; k < kWarps; ++k) {
+      const int n = wcnt[k][tid];
+      wcnt[k][tid] = run;
+      run += n;
+    }
+  }
+  __syncthreads();
+  if (live) {
+    const int dst = first[own] + wcnt[w][own] + rank;
+    p.req_rows[dst] = local;
+    p.req_pos[dst] = q;
+  }
+}
+
 __global__ void compress_kernel(const int64_t* __restrict__ raw, int64_t n,
                                 const int64_t* __restrict__ lookup, int64_t raw_vocab,
                                 int64_t* __restrict__ out, uint32_t* status) {
@@ -305,6 +418,24 @@ cudaError_t launch_compress(const int64_t* raw, int64_t n, const int64_t* lookup
   int cap = num_sms() * 8;
   if (blocks > cap) blocks = cap;
   launch_k(compress_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, raw, n, lookup, raw_vocab, out, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_route(const ShardRouteParams& p0, cudaStream_t s) {
+  ShardRouteParams p = p0;
+  HashParams& h = p.g.h;
+  if (p.n_shards < 1 || p.n_shards > ENGRAM_MAX_SHARDS) return cudaErrorInvalidValue;
+  const int64_t total = static_cast<int64_t>(h.B) * h.T * h.nh;
+  if (total <= 0) return cudaSuccess;
+  if (total + kShardChunk > INT32_MAX) return cudaErrorInvalidValue;   // 32-bit request ids
+  p.g.div_nh = make_fastdiv(static_cast<uint32_t>(h.nh));
+  p.g.div_J = make_fastdiv(static_cast<uint32_t>(h.J));
+  p.g.div_T = make_fastdiv(static_cast<uint32_t>(h.T));
+  p.div_shards = make_fastdiv(static_cast<uint32_t>(p.n_shards));
+  p.n_blk = static_cast<int32_t>((total + kShardChunk - 1) / kShardChunk);
+  launch_k(shard_count_kernel, dim3(static_cast<unsigned>(p.n_blk)), dim3(kShardChunk), 0, s, p);
+  launch_k(shard_scan_kernel, dim3(static_cast<unsigned>(p.n_shards)), dim3(1024), 0, s, p);
+  launch_k(shard_scatter_kernel, dim3(static_cast<unsigned>(p.n_blk)), dim3(kShardChunk), 0, s, p);
   return cudaGetLastError();
 }
 

@@ -51,6 +51,7 @@ extern "C" {
 #define ENGRAM_MAX_HC 8       /* hyper-connection branches */
 #define ENGRAM_MAX_CONV_K 8   /* short-conv kernel length */
 #define ENGRAM_MAX_LAYERS 4   /* Engram layers gathered in one engram_gather_ids_layers call */
+#define ENGRAM_MAX_SHARDS 64  /* devices one table may be sharded over (engram_shard_*) */
 
 typedef enum {
   ENGRAM_OK = 0,
@@ -293,6 +294,60 @@ engram_status engram_gather_ids_layers(const engram_config* cfg, const engram_we
                                        int32_t n_layers, const int64_t* ids, int32_t B, int32_t T,
                                        const int64_t* history, void* const* e, uint32_t* dev_status,
                                        engram_stream stream);
+
+/* ---- a table sharded over several devices ------------------------------
+ * The explainer page (§4.4) shards the tables across GPUs in training and
+ * collects the active rows with an All-to-All.  Split used here: shard r of
+ * n_shards holds the stacked table's rows r, r + n_shards, r + 2 n_shards, ...
+ * (engram_shard_rows of them), i.e. row -> shard row % n_shards, local row
+ * row / n_shards.  One gather of e then runs as
+ *   engram_shard_route  (this device's ids -> requests grouped by shard)
+ *   all-to-all          (counts, then the requested local rows)
+ *   engram_shard_serve  (on every device: the rows asked of its shard)
+ *   all-to-all          (the rows back, in request order)
+ *   engram_shard_place  (received rows -> their rows of e)
+ * and gives e bit for bit as engram_gather_ids on the whole table.  The
+ * exchanges are the caller's (NCCL over NVLink); these calls do the rest. */
+
+/* Rows held by shard `shard` of a table of total_rows rows split over
+ * n_shards; -1 for arguments out of range.  Host only. */
+int64_t engram_shard_rows(int64_t total_rows, int32_t n_shards, int32_t shard);
+
+/* DEVICE scratch bytes engram_shard_route needs for B x T ids. */
+size_t engram_shard_route_workspace_size(const engram_config* cfg, int32_t B, int32_t T, int32_t n_shards);
+
+/* The requests of the gather of e for ids: every row q = m*nh + h of e
+ * (hash as in engram_gather_ids) asks shard row % n_shards for local row
+ * row / n_shards.  Outputs, DEVICE, grouped by shard (shard 0 first) and in
+ * increasing q within a shard: counts [n_shards] int64 (requests per shard),
+ * req_rows [B*T*nh] int64 (the local row asked for), req_pos [B*T*nh] int32
+ * (the row q of e it fills).  weights: row_offsets, primes, multipliers,
+ * lookup, raw_vocab and total_rows (of the WHOLE table) are used; table is not
+ * read and may be NULL.  ws: DEVICE scratch of
+ * engram_shard_route_workspace_size bytes, 256-byte aligned.  n_shards in
+ * [1, ENGRAM_MAX_SHARDS]; B*T*nh < 2^31.  Out-of-range ids set
+ * ENGRAM_STATUS_ID_RANGE and hash as pad_id. */
+engram_status engram_shard_route(const engram_config* cfg, const engram_weights* weights, const int64_t* ids,
+                                 int32_t B, int32_t T, const int64_t* history, int32_t n_shards, int64_t* counts,
+                                 int64_t* req_rows, int32_t* req_pos, void* ws, size_t ws_bytes,
+                                 uint32_t* dev_status, engram_stream stream);
+
+/* The rows asked of this device's shard: out[k] = shard[req_rows[k]].
+ * shard: DEVICE [shard_rows, Dh] in cfg's dtype, 16-byte aligned (rows a
+ * multiple of 16 bytes); req_rows: DEVICE int64 [n]; out: DEVICE [n, Dh].  A
+ * request outside [0, shard_rows) writes a zero row and sets
+ * ENGRAM_STATUS_ROW_RANGE. */
+engram_status engram_shard_serve(const engram_config* cfg, const void* shard, int64_t shard_rows,
+                                 const int64_t* req_rows, int64_t n, void* out, uint32_t* dev_status,
+                                 engram_stream stream);
+
+/* The received rows to their rows of e: e[req_pos[k]] = got[k].  got: DEVICE
+ * [n, Dh] (the rows in engram_shard_route's request order); req_pos: DEVICE
+ * int32 [n]; e: DEVICE [n_e, Dh] (n_e = B*T*nh rows of Dh: the layout of
+ * engram_gather_ids' e).  A position outside [0, n_e) is skipped and sets
+ * ENGRAM_STATUS_ROW_RANGE. */
+engram_status engram_shard_place(const engram_config* cfg, const void* got, const int32_t* req_pos, int64_t n,
+                                 void* e, int64_t n_e, uint32_t* dev_status, engram_stream stream);
 
 /* The rest of engram_forward (a5-a9) on rows gathered by engram_gather_ids:
  * y = the same result engram_forward gives for those ids (bit for bit on the

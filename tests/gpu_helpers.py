@@ -2,7 +2,7 @@
 oracle run on the same inputs (whole pass, or sampled positions with rows
 fetched from the device tables), and the tolerance rule.
 
-Tolerance (spec rule, per output tensor): max |y - y_ref| must not
+Tolerance (the bound set for this pass, per output tensor): max |y - y_ref| must not
 exceed tol * max |y_ref| with tol = 1e-4 for float32 and 2e-2 for bfloat16,
 y_ref from the float64 oracle on the same (bf16-valued) inputs.
 """
@@ -74,3 +74,16 @@ def sample_positions(B: int, T: int, dil: int, n_random: int, seed: int = 0):
 
 def device_params(w: W.Workload, device="cuda"):
     return W.make_params(w, device)
+
+
+def make_layer(p, table=None):
+    """EngramLayer of a workloads.Params (table: another copy of the table)."""
+    from hashed_gram_conditional_hash_b200 import EngramLayer
+    w = p.w
+    return EngramLayer(orders=w.orders, heads_per_order=w.heads_per_order, row_dim=w.row_dim,
+                       hidden=w.hidden, hc_mult=w.hc_mult, conv_kernel=w.conv_kernel,
+                       dilation=w.dil, pad_id=w.pad_id, vocab=w.vocab,
+                       table=p.table if table is None else table, row_offsets=p.offsets,
+                       primes=p.primes, multipliers=p.mult, w_value=p.w_value, w_key=p.w_key,
+                       norm_key=p.norm_key, norm_query=p.norm_query, conv_w=p.conv_w,
+                       lookup=p.lookup, rms_eps=w.rms_eps, gate_eps=w.gate_eps)

@@ -13,7 +13,7 @@ from hashed_gram_conditional_hash_b200 import EngramLayer
 from hashed_gram_conditional_hash_b200 import _lib as L
 from hashed_gram_conditional_hash_b200 import workloads as W
 
-from gpu_helpers import device_params, oracle_ids
+from gpu_helpers import device_params, make_layer, oracle_ids
 from oracle import engram_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -21,14 +21,7 @@ DEV = "cuda"
 
 
 def _layer(p, table=None):
-    w = p.w
-    return EngramLayer(orders=w.orders, heads_per_order=w.heads_per_order, row_dim=w.row_dim,
-                       hidden=w.hidden, hc_mult=w.hc_mult, conv_kernel=w.conv_kernel,
-                       dilation=w.dil, pad_id=w.pad_id, vocab=w.vocab,
-                       table=p.table if table is None else table, row_offsets=p.offsets,
-                       primes=p.primes, multipliers=p.mult, w_value=p.w_value, w_key=p.w_key,
-                       norm_key=p.norm_key, norm_query=p.norm_query, conv_w=p.conv_w,
-                       lookup=p.lookup, rms_eps=w.rms_eps, gate_eps=w.gate_eps)
+    return make_layer(p, table)
 
 
 CASES = [W.small_workload(), W.small_workload(B=2, T=130, hidden=512, hc_mult=4, orders=(2, 3, 4)),
