@@ -404,22 +404,6 @@ template <> struct LaneRow<8> {
   static __device__ __forceinline__ void unpack(const raw_t& w, float2 (&v)[4]) { Pair8<uint16_t>::unpack(w, v); }
   static __device__ __forceinline__ void store(uint16_t* p, const float2 (&v)[4]) { Pair8<uint16_t>::store(p, v); }
 };
-template <> struct LaneRow<4> {
-  using raw_t = uint2;
-  static __device__ __forceinline__ raw_t lds(uint32_t a) {
-    uint2 r;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a));
-    return r;
-  }
-  static __device__ __forceinline__ void unpack(const raw_t& w, float2 (&v)[2]) {
-    v[0] = make_float2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
-    v[1] = make_float2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
-  }
-  static __device__ __forceinline__ void store(uint16_t* p, const float2 (&v)[2]) {
-    *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0].x, v[0].y), pack_bf16x2(v[1].x, v[1].y));
-  }
-};
-
 // The K = 4 taps of CPL consecutive channels (4*CPL contiguous bf16 values,
 // channel-major) as w2[pair][tap] = (tap of channel 2 pair, of channel 2 pair + 1).
 template <int CPL>

@@ -154,21 +154,22 @@ __device__ __forceinline__ void hash_gather_body(const HashGatherParams& g) {
   const char* tab = static_cast<const char*>(g.table);
   if (CH > 0) {
     // piece i of the warp's rows is row i / CH, 16-byte column i % CH
-    constexpr int kPer = ROWS * (CH > 0 ? CH : 1) / 32;   // pieces per lane
+    constexpr int kCh = CH > 0 ? CH : 1;             // (this branch only runs with CH > 0)
+    constexpr int kPer = ROWS * kCh / 32;            // pieces per lane
     int4 v[kPer];
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int i = u * 32 + lane;
-      const int r = i / CH;
+      const int r = i / kCh;
       const int64_t src = __shfl_sync(0xffffffffu, row, r);
       if (q0 + r < total)
-        v[u] = ld_row_piece<HOSTMEM>(reinterpret_cast<const int4*>(tab + src * (CH * 16)) + (i - r * CH));
+        v[u] = ld_row_piece<HOSTMEM>(reinterpret_cast<const int4*>(tab + src * (kCh * 16)) + (i - r * kCh));
     }
-    int4* out = static_cast<int4*>(g.e) + static_cast<int64_t>(q0) * CH;
+    int4* out = static_cast<int4*>(g.e) + static_cast<int64_t>(q0) * kCh;
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int i = u * 32 + lane;
-      if (q0 + i / CH < total) out[i] = v[u];
+      if (q0 + i / kCh < total) out[i] = v[u];
     }
     return;
   }
