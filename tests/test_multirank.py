@@ -42,7 +42,7 @@ def _rank_main(rank, world, port, per_rank_ms, out):
 def test_max_over_ranks_and_job_throughput_two_gloo_ranks():
     world = 2
     per_rank_ms = [[5.0, 1.0, 9.0], [7.5, 0.5, 9.5]]
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_rank_main, args=(world, _free_port(), per_rank_ms, out), nprocs=world,
                            join=True, start_method="spawn")

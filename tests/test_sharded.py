@@ -105,7 +105,7 @@ def _rank_main(rank, world, port, out):
 
 @pytest.mark.parametrize("world", [2, 3])
 def test_sharded_gather_exchange_over_gloo_ranks(world):
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True,
                            start_method="spawn")
