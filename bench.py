@@ -203,6 +203,26 @@ def algorithmic(w):
     }
 
 
+def pass_roofline(w, tokens_step, step_s, tc_peak_tflops, hbm_gbs):
+    """The whole pass against its own roofline: the bytes the method must move
+    (ids, gathered rows, hidden read, Y written, the weights once per step;
+    in decode also the three V-ring taps read and the step's V row written)
+    and the projection flops; t = max(bytes / HBM peak, flops / tensor peak),
+    frac = t / the measured step time."""
+    es = w.elem_bytes
+    per_tok = 8 + w.E * es + 2 * w.hc_mult * w.hidden * es
+    if w.decode_calls:
+        per_tok += 4 * w.hidden * es
+    weights = (1 + w.hc_mult) * w.hidden * w.E * es
+    nbytes = per_tok * tokens_step + weights
+    flops = algorithmic(w)["proj_flops"] * tokens_step
+    t_hbm = nbytes / (hbm_gbs * 1e9)
+    t_tc = flops / (tc_peak_tflops * 1e12)
+    return {"bytes_per_step": nbytes, "flops_per_step": flops, "t_hbm_us": t_hbm * 1e6,
+            "t_tensor_us": t_tc * 1e6, "bound": "tensor" if t_tc >= t_hbm else "hbm",
+            "frac": max(t_hbm, t_tc) / step_s}
+
+
 def max_over_ranks(t, world):
     """Element-wise max over ranks of a float64 tensor of per-rank timings
     (on the device of the process group's backend); identity for one rank."""
@@ -351,6 +371,7 @@ def run_ours(args, rank, world, device):
                      "frac": proj_tflops / tc_peak, "peak_kind": "%s bf16 %s" % (peak_kind, "sustained" if sustained else "burst"),
                      "traffic": kernel_traffic(kname, w.name),
                      "flops_per_launch": a["proj_flops"] * tokens_step},
+        "pass_roofline": pass_roofline(w, tokens_step, t_step / K / 1e3, tc_peak, peaks["hbm_gbs"]),
         "stages": stages,
         "clocks": clk,
         "gpu_launches": int(launches),
@@ -593,6 +614,35 @@ def run_sharded(args, layer, p, w, device):
                     "direction, not measured" % PEER_COPY_GBS}
 
 
+def hbm_rates(device):
+    """Write-only, read-only and copy rates of HBM on 1 GiB buffers (torch fill,
+    sum and copy kernels; median of 20 launches by CUDA events): the read and
+    write sides of the roofline of kernels whose traffic is mostly one way."""
+    n = 1 << 30
+    a = torch.empty(n, dtype=torch.uint8, device=device)
+    b = torch.empty_like(a)
+    out = torch.empty((), dtype=torch.int64, device=device)
+
+    def med_ms(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+        for e0, e1 in ev:
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return sorted(x.elapsed_time(y) for x, y in ev)[10]
+
+    a.fill_(1)
+    t_w = med_ms(lambda: a.fill_(2))
+    t_r = med_ms(lambda: torch.sum(a.view(torch.int64), dim=0, out=out))
+    t_c = med_ms(lambda: b.copy_(a))
+    return {"write_only_gbs": n / t_w / 1e6, "read_only_gbs": n / t_r / 1e6, "copy_gbs": 2 * n / t_c / 1e6,
+            "bytes": n, "note": "torch fill_ / sum / copy_ on 1 GiB, median of 20 launches"}
+
+
 def run_reference(args):
     """The reference arm: the float64 oracle on the host cores, K timed steps
     of a bounded sample each, sized so that warm-up + steps take ~2 minutes."""
@@ -637,6 +687,8 @@ def main():
                     help="decode workload: number of distinct calls drawn (default: all 256)")
     ap.add_argument("--offload", action="store_true",
                     help="also measure tables resident in pinned host memory (prefill workloads)")
+    ap.add_argument("--hbm-rates", action="store_true",
+                    help="also measure HBM write-only, read-only and copy rates (1 GiB torch kernels)")
     ap.add_argument("--sharded", type=int, default=0,
                     help="also time the device steps of a gather from a table sharded over this many GPUs")
     args = ap.parse_args()
@@ -662,6 +714,8 @@ def main():
             res["e2e"] = run_e2e(args, layer, p, w, device, world)
         if args.offload and not w.decode_calls:
             res["offload"] = run_offload(args, layer, p, w, device)
+        if args.hbm_rates:
+            res["hbm_rates"] = hbm_rates(device)
         if args.sharded and not w.decode_calls:
             res["sharded"] = run_sharded(args, layer, p, w, device)
         del layer, p

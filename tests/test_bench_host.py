@@ -1,0 +1,33 @@
+"""Host arithmetic of bench.py: the whole-pass roofline counts the bytes the
+method must move and the projection flops (per token: the id, the gathered
+rows, hidden read, Y written; the weights once per step; in decode also three
+V-ring taps read and one V row written)."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from hashed_gram_conditional_hash_b200 import workloads as W  # noqa: E402
+
+
+def test_pass_roofline_model_shaped_counts():
+    w = W.CONFIGS["model_bf16"]             # B=4, T=2048, E=1024, H=1024, hc=4, bf16
+    tok = 4 * 2048
+    r = bench.pass_roofline(w, tok, 100e-6, 1661.2, 6550.4)
+    assert r["bytes_per_step"] == tok * (8 + 1024 * 2 + 2 * 4 * 1024 * 2) + 5 * 1024 * 1024 * 2
+    assert r["flops_per_step"] == 2 * 1024 * 1024 * 5 * tok
+    assert r["bound"] == "tensor"
+    assert r["t_tensor_us"] == pytest.approx(2 * 1024 * 1024 * 5 * tok / 1661.2e12 * 1e6)
+    assert r["frac"] == pytest.approx(r["t_tensor_us"] / 100.0)
+
+
+def test_pass_roofline_decode_adds_ring_traffic():
+    w = W.CONFIGS["decode_bf16"]            # 1024 sequences x 1 token, E=1536, H=2048, hc=4
+    r = bench.pass_roofline(w, 1024, 64e-6, 1661.2, 6550.4)
+    per_tok = 8 + 1536 * 2 + 2 * 4 * 2048 * 2 + 4 * 2048 * 2
+    assert r["bytes_per_step"] == 1024 * per_tok + 5 * 2048 * 1536 * 2
+    assert r["t_hbm_us"] == pytest.approx(r["bytes_per_step"] / 6550.4e9 * 1e6)
