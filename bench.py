@@ -166,12 +166,17 @@ def oracle_tokens_for(w, seconds: float, nthreads: int) -> int:
 
 
 def cpu_baseline(w, budget_s: float):
+    """The oracle on all host cores (the reported value) and on one core."""
     nthreads = os.cpu_count() or 1
     n, run = oracle_sample(w, oracle_tokens_for(w, budget_s, nthreads), nthreads)
     dt = run()
+    n1, run1 = oracle_sample(w, oracle_tokens_for(w, budget_s / 4, 1), 1)
+    dt1 = run1()
     return {"value": n / dt, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+            "single_thread_value": n1 / dt1,
             "sample": "%d positions (whole sequences) of a workload with the shapes and "
-                      "distributions of %s, whole pass from ids, float64, %.1f s" % (n, w.name, dt)}
+                      "distributions of %s, whole pass from ids, float64, %.1f s; one thread: %d "
+                      "positions, %.1f s" % (n, w.name, dt, n1, dt1)}
 
 
 # ---------------------------------------------------------------- GPU arm
