@@ -105,3 +105,84 @@ def test_short_conv_rejects_aliasing():
     rc = L.lib().engram_short_conv(C.byref(cfg), C.c_void_p(256), 1, 4, C.c_void_p(512), None,
                                    C.c_void_p(256), None)
     assert rc == 1
+
+
+# ---- the split pass, several layers and the sharded table: host-side checks
+P = C.c_void_p
+
+
+def _weights():
+    w = L.EngramWeights()
+    w.table = 256
+    w.total_rows = 1000
+    return w
+
+
+def test_gather_ids_layers_rejects_layer_counts():
+    cfg = _cfg()
+    w = _weights()
+    arr = (C.POINTER(L.EngramWeights) * 1)(C.pointer(w))
+    e = (P * 1)(256)
+    for n in (0, L.MAX_LAYERS + 1):
+        assert L.lib().engram_gather_ids_layers(C.byref(cfg), arr, n, P(256), 2, 8, None, e, None, None) == 1
+        assert "n_layers" in L.last_error()
+    assert L.lib().engram_gather_ids_layers(C.byref(cfg), None, 1, P(256), 2, 8, None, e, None, None) == 1
+
+
+@pytest.mark.parametrize("n_shards", [0, L.MAX_SHARDS + 1])
+def test_shard_route_rejects_shard_counts(n_shards):
+    cfg = _cfg()
+    w = _weights()
+    rc = L.lib().engram_shard_route(C.byref(cfg), C.byref(w), P(256), 2, 8, None, n_shards, P(256), P(256),
+                                    P(256), P(256), 1 << 20, None, None)
+    assert rc == 1 and "n_shards" in L.last_error()
+
+
+def test_shard_route_rejects_missing_or_small_workspace():
+    cfg = _cfg()
+    w = _weights()
+    need = L.engram_shard_route_workspace_size(cfg, 2, 8, 4)
+    assert need > 0
+    args = lambda counts, ws, nbytes: (C.byref(cfg), C.byref(w), P(256), 2, 8, None, 4, counts, P(256), P(256),
+                                       ws, nbytes, None, None)
+    assert L.lib().engram_shard_route(*args(None, P(256), need)) == 1          # counts NULL
+    assert L.lib().engram_shard_route(*args(P(256), None, need)) == 1          # ws NULL
+    assert L.lib().engram_shard_route(*args(P(256), P(272), need)) == 1        # ws not 256-byte aligned
+    assert "aligned" in L.last_error()
+    assert L.lib().engram_shard_route(*args(P(256), P(256), need - 1)) == 1    # too small
+    assert "too small" in L.last_error()
+    big = _cfg(heads_per_order=32)                                            # B*T*nh >= 2^31
+    assert L.lib().engram_shard_route(C.byref(big), C.byref(w), P(256), 1 << 20, 1 << 10, None, 2, P(256),
+                                      P(256), P(256), P(256), 1 << 20, None, None) == 2
+
+
+def test_shard_serve_and_place_reject_bad_arguments():
+    cfg = _cfg()
+    lib = L.lib()
+    assert lib.engram_shard_serve(C.byref(cfg), P(256), 10, P(256), -1, P(256), None, None) == 1
+    assert lib.engram_shard_serve(C.byref(cfg), None, 10, P(256), 4, P(256), None, None) == 1
+    assert lib.engram_shard_serve(C.byref(cfg), P(256), 10, P(256), 4, P(264), None, None) == 1   # misaligned out
+    narrow = _cfg(row_dim=2)                                                  # 4-byte rows
+    assert lib.engram_shard_serve(C.byref(narrow), P(256), 10, P(256), 4, P(256), None, None) == 2
+    assert lib.engram_shard_place(C.byref(cfg), P(256), P(256), -1, P(256), 8, None, None) == 1
+    assert lib.engram_shard_place(C.byref(cfg), P(256), None, 4, P(256), 8, None, None) == 1
+    assert lib.engram_shard_place(C.byref(cfg), P(264), P(256), 4, P(256), 8, None, None) == 1    # misaligned got
+    assert lib.engram_shard_place(C.byref(narrow), P(256), P(256), 4, P(256), 8, None, None) == 2
+    # nothing to do is not an error, and launches nothing
+    assert lib.engram_shard_serve(C.byref(cfg), None, 0, None, 0, None, None, None) == 0
+    assert lib.engram_shard_place(C.byref(cfg), None, None, 0, None, 0, None, None) == 0
+
+
+def test_forward_gathered_rejects_null_misaligned_and_small_workspace():
+    cfg = _cfg()
+    w = L.EngramWeights()
+    for f in ("w_value", "w_key", "norm_key", "norm_query", "conv_w"):
+        setattr(w, f, 256)
+    need = L.engram_forward_workspace_size(cfg, 2, 8)
+    lib = L.lib()
+    ok = dict(e=P(256), hidden=P(256), y=P(256), ws=P(256), n=need)
+    call = lambda **kw: lib.engram_forward_gathered(C.byref(cfg), C.byref(w), kw["e"], 2, 8, kw["hidden"], kw["y"],
+                                                    kw["ws"], kw["n"], None, None)
+    assert call(**dict(ok, e=None)) == 1
+    assert call(**dict(ok, y=P(264))) == 1
+    assert call(**dict(ok, n=need - 1)) == 1 and "too small" in L.last_error()
