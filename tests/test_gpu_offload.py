@@ -106,3 +106,20 @@ def test_gather_ids_layers_equals_per_layer_gathers():
     # and the rows reach each layer's own forward
     y0 = layers[0].forward_gathered(e[0], ps[0].hidden)
     assert torch.equal(y0, layers[0].forward(ids, ps[0].hidden))
+
+
+def test_gather_ids_layers_with_history_continues_sequences():
+    base = W.small_workload(B=3, T=40, orders=(2, 3, 4))
+    ps = [device_params(base.replace(layer_id=1, seed=31)), device_params(base.replace(layer_id=4, seed=32))]
+    layers = [_layer(p) for p in ps]
+    ids = ps[0].ids
+    hist = ids[:, 17:20].contiguous()                 # the 3 ids before position 20
+    tail = ids[:, 20:].contiguous()
+    E = base.nh * base.row_dim
+    e = [torch.empty((base.B * 20, E), dtype=ps[0].table.dtype, device=DEV) for _ in layers]
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    L.engram_gather_ids_layers(layers[0].cfg, [l.weights for l in layers], tail, e, history=hist, dev_status=st)
+    assert L.engram_read_status(st) == 0
+    for layer, e_l in zip(layers, e):
+        full = layer.gather_ids(ids)
+        assert torch.equal(e_l.view(base.B, -1, E), full.view(base.B, base.T, E)[:, 20:])
