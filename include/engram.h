@@ -324,9 +324,14 @@ size_t engram_shard_route_workspace_size(const engram_config* cfg, int32_t B, in
  * (the row q of e it fills).  weights: row_offsets, primes, multipliers,
  * lookup, raw_vocab and total_rows (of the WHOLE table) are used; table is not
  * read and may be NULL.  ws: DEVICE scratch of
- * engram_shard_route_workspace_size bytes, 256-byte aligned.  n_shards in
- * [1, ENGRAM_MAX_SHARDS]; B*T*nh < 2^31.  Out-of-range ids set
- * ENGRAM_STATUS_ID_RANGE and hash as pad_id. */
+ * engram_shard_route_workspace_size bytes, 256-byte aligned.  ids: DEVICE
+ * [B, T], 16-byte aligned; history: DEVICE [B, max_n - 1] or NULL, as in
+ * engram_gather_ids.  Every buffer is the caller's.  n_shards in
+ * [1, ENGRAM_MAX_SHARDS]; B*T*nh < 2^31.  B*T == 0 writes zero counts.
+ * Errors: ENGRAM_ERR_INVALID_ARG (n_shards out of range, a NULL or misaligned
+ * pointer, a workspace too small), ENGRAM_ERR_UNSUPPORTED (B*T*nh or
+ * total_rows >= 2^31, rows not a multiple of 16 bytes), both before any
+ * launch.  Out-of-range ids set ENGRAM_STATUS_ID_RANGE and hash as pad_id. */
 engram_status engram_shard_route(const engram_config* cfg, const engram_weights* weights, const int64_t* ids,
                                  int32_t B, int32_t T, const int64_t* history, int32_t n_shards, int64_t* counts,
                                  int64_t* req_rows, int32_t* req_pos, void* ws, size_t ws_bytes,
@@ -334,8 +339,11 @@ engram_status engram_shard_route(const engram_config* cfg, const engram_weights*
 
 /* The rows asked of this device's shard: out[k] = shard[req_rows[k]].
  * shard: DEVICE [shard_rows, Dh] in cfg's dtype, 16-byte aligned (rows a
- * multiple of 16 bytes); req_rows: DEVICE int64 [n]; out: DEVICE [n, Dh].  A
- * request outside [0, shard_rows) writes a zero row and sets
+ * multiple of 16 bytes); req_rows: DEVICE int64 [n]; out: DEVICE [n, Dh],
+ * 16-byte aligned; all the caller's.  n == 0 does nothing.  Errors:
+ * ENGRAM_ERR_INVALID_ARG (n < 0, a NULL or misaligned pointer, a shard in host
+ * memory), ENGRAM_ERR_UNSUPPORTED (rows not a multiple of 16 bytes), before any
+ * launch.  A request outside [0, shard_rows) writes a zero row and sets
  * ENGRAM_STATUS_ROW_RANGE. */
 engram_status engram_shard_serve(const engram_config* cfg, const void* shard, int64_t shard_rows,
                                  const int64_t* req_rows, int64_t n, void* out, uint32_t* dev_status,
@@ -344,7 +352,10 @@ engram_status engram_shard_serve(const engram_config* cfg, const void* shard, in
 /* The received rows to their rows of e: e[req_pos[k]] = got[k].  got: DEVICE
  * [n, Dh] (the rows in engram_shard_route's request order); req_pos: DEVICE
  * int32 [n]; e: DEVICE [n_e, Dh] (n_e = B*T*nh rows of Dh: the layout of
- * engram_gather_ids' e).  A position outside [0, n_e) is skipped and sets
+ * engram_gather_ids' e); got and e 16-byte aligned; all the caller's.  n == 0
+ * does nothing.  Errors: ENGRAM_ERR_INVALID_ARG (n or n_e < 0, a NULL or
+ * misaligned pointer), ENGRAM_ERR_UNSUPPORTED (rows not a multiple of 16
+ * bytes), before any launch.  A position outside [0, n_e) is skipped and sets
  * ENGRAM_STATUS_ROW_RANGE. */
 engram_status engram_shard_place(const engram_config* cfg, const void* got, const int32_t* req_pos, int64_t n,
                                  void* e, int64_t n_e, uint32_t* dev_status, engram_stream stream);
