@@ -288,8 +288,13 @@ engram_status engram_gather_ids(const engram_config* cfg, const engram_weights* 
  * layers[l]: the weights of layer l (table, total_rows, row_offsets, primes,
  * multipliers, lookup, raw_vocab as in engram_gather_ids); e[l]: DEVICE
  * [B*T, nh*Dh] output of layer l.  All layers share cfg (orders, heads, row
- * width, dtype).  n_layers in [1, ENGRAM_MAX_LAYERS].  The rows of each layer
- * are bit for bit those engram_gather_ids gives for it. */
+ * width, dtype).  layers and e are HOST arrays of n_layers pointers; ids and
+ * every e[l] are 16-byte aligned; each layer's table may be device or pinned
+ * host memory; all buffers are the caller's.  n_layers in
+ * [1, ENGRAM_MAX_LAYERS].  Errors as engram_gather_ids (and
+ * ENGRAM_ERR_INVALID_ARG for n_layers out of range or NULL arrays), before any
+ * launch.  The rows of each layer are bit for bit those engram_gather_ids
+ * gives for it. */
 engram_status engram_gather_ids_layers(const engram_config* cfg, const engram_weights* const* layers,
                                        int32_t n_layers, const int64_t* ids, int32_t B, int32_t T,
                                        const int64_t* history, void* const* e, uint32_t* dev_status,
@@ -366,7 +371,11 @@ engram_status engram_shard_place(const engram_config* cfg, const void* got, cons
  * caller that keeps no state).  e: DEVICE [B*T, nh*Dh]; hidden, y: DEVICE
  * [B, T, hc, H]; ws: DEVICE scratch of engram_forward_workspace_size(cfg, B, T)
  * bytes, 256-byte aligned.  Uses weights->w_value, w_key, norm_key,
- * norm_query, conv_w. */
+ * norm_query, conv_w.  All pointers 16-byte aligned and the caller's.
+ * Errors: ENGRAM_ERR_INVALID_ARG (a NULL or misaligned pointer, a workspace too
+ * small), ENGRAM_ERR_UNSUPPORTED (hidden not a multiple of 64, rows not a
+ * multiple of 16 bytes), before any launch; a bounded pipeline wait that runs
+ * out sets ENGRAM_STATUS_TIMEOUT in *dev_status. */
 engram_status engram_forward_gathered(const engram_config* cfg, const engram_weights* weights, const void* e,
                                       int32_t B, int32_t T, const void* hidden, void* y, void* ws,
                                       size_t ws_bytes, uint32_t* dev_status, engram_stream stream);
