@@ -60,6 +60,9 @@ def _doubles(w, p):
     offsets = np.asarray(p.offsets)
 
     def route(cfg, weights, ids, R, counts, req_rows, req_pos, ws, history=None, dev_status=None, stream=None):
+        if ids.numel() == 0:
+            counts.zero_()
+            return
         idx = O.ngram_hash(ids.numpy(), w.orders, w.heads_per_order, p.mult, p.primes, w.pad_id)
         c, rr, rp = O.shard_route((idx + offsets[None, None, :]).reshape(-1), R)
         counts.copy_(torch.from_numpy(c))
@@ -70,12 +73,14 @@ def _doubles(w, p):
         out.copy_(shard[req_rows])
 
     def place(cfg, got, req_pos, e, n_e, dev_status=None, stream=None):
+        if req_pos.numel() == 0:                 # as the library: nothing to place
+            return
         e.view(n_e, -1)[req_pos.long()] = got
 
     return route, serve, place
 
 
-def _rank_main(rank, world, port, out):
+def _rank_main(rank, world, port, out, empty_rank=-1):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     from hashed_gram_conditional_hash_b200 import sharded
@@ -83,6 +88,8 @@ def _rank_main(rank, world, port, out):
     w = W.small_workload(B=2, T=50, orders=(2, 3, 4), seed=30 + rank)   # each rank its own ids
     p = W.make_params(w.replace(seed=30), "cpu")                          # one table for all ranks
     ids = W.make_params(w, "cpu").ids
+    if rank == empty_rank:                                                  # no ids, still serves its shard
+        ids = ids[:, :0].contiguous()
     Lr.engram_shard_route, Lr.engram_shard_serve, Lr.engram_shard_place = _doubles(w, p)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -95,6 +102,9 @@ def _rank_main(rank, world, port, out):
         sg = sharded.ShardedGather(cfg, shard, total_rows=p.table.shape[0], row_offsets=p.offsets,
                                    primes=p.primes, multipliers=p.mult)
         e = sg.gather_ids(ids)
+        if ids.numel() == 0:
+            out[rank] = e.shape[0] == 0, int(e.shape[0])
+            return
         idx = O.ngram_hash(ids.numpy(), w.orders, w.heads_per_order, p.mult, p.primes, w.pad_id)
         ref = O.gather(full, p.offsets, idx.reshape(-1, w.nh))
         got = e.view(torch.int16).numpy() if e.dtype == torch.bfloat16 else e.numpy()
@@ -103,15 +113,15 @@ def _rank_main(rank, world, port, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_sharded_gather_exchange_over_gloo_ranks(world):
+@pytest.mark.parametrize("world,empty_rank", [(2, -1), (3, -1), (2, 1)])
+def test_sharded_gather_exchange_over_gloo_ranks(world, empty_rank):
     with mp.get_context("spawn").Manager() as m:
         out = m.dict()
-        mp.start_processes(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True,
+        mp.start_processes(_rank_main, args=(world, _free_port(), out, empty_rank), nprocs=world, join=True,
                            start_method="spawn")
         res = dict(out)
     assert sorted(res) == list(range(world))
     for rank in range(world):
         ok, rows = res[rank]
         assert ok, "rank %d: e differs from the gather of the whole table" % rank
-        assert rows == 2 * 50
+        assert rows == (0 if rank == empty_rank else 2 * 50)
