@@ -186,3 +186,11 @@ def test_forward_gathered_rejects_null_misaligned_and_small_workspace():
     assert call(**dict(ok, e=None)) == 1
     assert call(**dict(ok, y=P(264))) == 1
     assert call(**dict(ok, n=need - 1)) == 1 and "too small" in L.last_error()
+
+
+def test_binding_declares_every_signature():
+    # ctypes passes undeclared arguments as C ints: every entry point the
+    # header declares must have its argument and result types set
+    lib = L.lib()
+    missing = [n for n in _declared() if getattr(lib, n).argtypes is None]
+    assert not missing, missing
