@@ -31,3 +31,16 @@ def test_pass_roofline_decode_adds_ring_traffic():
     per_tok = 8 + 1536 * 2 + 2 * 4 * 2048 * 2 + 4 * 2048 * 2
     assert r["bytes_per_step"] == 1024 * per_tok + 5 * 2048 * 1536 * 2
     assert r["t_hbm_us"] == pytest.approx(r["bytes_per_step"] / 6550.4e9 * 1e6)
+
+
+@pytest.mark.parametrize("name,tokens,total_bytes,total_flops", [
+    # per token 8 + 2E + 4·hc·H bytes, weights (1+hc)·H·E·2 once, 2·E·H·(1+hc) flops
+    ("large_table_bf16", 8 * 4096, 1.4824e9, 1.2885e12),
+    ("hbm_table_bf16", 16 * 4096, 4.6478e9, 5.4976e12),
+])
+def test_pass_roofline_large_workloads(name, tokens, total_bytes, total_flops):
+    w = W.CONFIGS[name]
+    r = bench.pass_roofline(w, tokens, 1e-3, 1661.2, 6550.4)
+    assert r["bytes_per_step"] == pytest.approx(total_bytes, rel=1e-3)
+    assert r["flops_per_step"] == pytest.approx(total_flops, rel=1e-3)
+    assert r["bound"] == "tensor"
