@@ -3,6 +3,8 @@
 // input and output buffers, a latency-critical loop where cudaMalloc/cudaFree
 // would synchronise the device).  It adds an entry point and changes nothing
 // in engram_forward, which it calls with the array as the workspace.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "engram_internal.cuh"
@@ -16,9 +18,46 @@ static __device__ __align__(256) unsigned char g_no_alloc_scratch[kScratchBytes]
 
 // Device address of the array per device.  In host code the array's name is
 // only a host-side stand-in, so the address must come from
-// cudaGetSymbolAddress, looked up once per device with that device current.
+// cudaGetSymbolAddress, looked up with that device current.  The address
+// belongs to the device's current context: after cudaDeviceReset (or any
+// other teardown of the primary context) the module is loaded again and the
+// array may move.  So each cached address is tagged with the unique id of
+// the context it was looked up in (cuCtxGetId; ids are never reused within a
+// process) and looked up again when the current context's id differs.
+struct Cached {
+  unsigned long long ctx_id = 0;
+  void* addr = nullptr;
+};
 std::mutex g_mu;
-void* g_scratch_addr[256] = {};
+Cached g_scratch[256];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context; false when there is no
+// current context yet or the driver offers no context ids.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool resolved = false;
+  if (!resolved) {  // (under g_mu)
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    cudaGetLastError();
+    resolved = true;
+  }
+  if (get_current == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 }  // namespace
 
@@ -44,15 +83,23 @@ extern "C" engram_status engram_forward_no_alloc(const engram_config* cfg,
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    unsigned long long ctx = 0;
+    const bool have_ctx = current_context_id(&ctx);
+    Cached& c = g_scratch[dev];
+    if (!have_ctx || c.addr == nullptr || c.ctx_id != ctx) {
       void* addr = nullptr;
       e = cudaGetSymbolAddress(&addr, g_no_alloc_scratch);
       if (e != cudaSuccess || addr == nullptr)
         return engram::set_error(ENGRAM_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s",
                                  cudaGetErrorString(e));
-      g_scratch_addr[dev] = addr;
+      // the lookup made the primary context current if it was not yet
+      c.addr = addr;
+      c.ctx_id = current_context_id(&ctx) ? ctx : 0;
+      if (c.ctx_id == 0) c.addr = nullptr;   // no context ids: look up again next call
+      scratch = addr;
+    } else {
+      scratch = c.addr;
     }
-    scratch = g_scratch_addr[dev];
   }
   return engram_forward(cfg, weights, ids, B, T, hidden, y, state, scratch, kScratchBytes,
                         dev_status, stream);

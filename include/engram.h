@@ -400,8 +400,11 @@ engram_status engram_forward_gathered(const engram_config* cfg, const engram_wei
  * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *
  * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture.  Every call on a device shares the one array and leaves its
+ * device current) and caches it, tagged with the current context's unique id;
+ * a call made in another context of that device (after cudaDeviceReset, say)
+ * looks it up again, as the array may have moved.  Make the first call in a
+ * context before any stream capture.  Every call on a device shares the one
+ * array and leaves its
  * contents behind (the pass writes every scratch byte it reads, so nothing
  * needs clearing); calls that overlap on the GPU, on different streams or
  * host threads, race on it and give undefined results. */
