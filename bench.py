@@ -3,12 +3,17 @@
 
 One step = one engram_forward over one batch of the workload (hash + row
 gather -> tcgen05 projection on CTA pairs + score partials -> gate -> gated
-value + short conv + residual), inputs resident in HBM.  Default workload: the bf16 model-shaped
-one (B=4, T=2048, 16 heads x 64 = 1024-d e_t, H=1024, hc=4).
+value + short conv + residual), inputs resident in HBM.  Default workload: the
+largest one that fits one GPU, the HBM-scale table (B=16, T=4096, 32 heads x
+2^22 rows x 64 bf16 = 17.2 GB of tables, H=4096, hc=4); --config selects the
+others (model_bf16, large_table_bf16, decode_bf16, tiny_f32).
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
-the launching stream; L2 is flushed (256 MB write) between steps outside the
-events; barrier + synchronize on both sides; the max over ranks is reported.
+the launching stream; between steps, outside the events, L2 is flushed (a
+256 MB write) and then drained (a 256 MB read of another buffer, so the
+flush's dirty lines are written back before the next step starts instead of
+during its first kernel); barrier + synchronize on both sides; the max over
+ranks is reported.
 Multi-GPU: one process per GPU, every rank runs its own replica of the
 workload (the pass has no cross-sequence exchange), scaling "weak".
 
@@ -110,10 +115,12 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- oracle (CPU)
-def oracle_sample(w, tokens: int, nthreads: int):
+def oracle_sample(w, tokens: int, nthreads: int, p=None):
     """Prepare the float64 oracle over the first `tokens` positions of
     sequence 0 of a workload of the same shapes and distributions (whole pass
-    from ids, host cores).  Returns (n, run) where run() -> seconds."""
+    from ids, host cores).  Returns (n, run) where run() -> seconds.  For a
+    workload whose tables are drawn on the device, p (its device Params) may
+    be passed in to avoid drawing them again."""
     from hashed_gram_conditional_hash_b200 import workloads as W
     from oracle import engram_oracle as O
     n = max(1, min(tokens, w.B * w.seq_len))
@@ -137,7 +144,8 @@ def oracle_sample(w, tokens: int, nthreads: int):
             return time.perf_counter() - t0
         return n, run
     # tables drawn on the device: the oracle receives the rows it needs
-    p = W.make_params(w, "cuda")
+    if p is None:
+        p = W.make_params(w, "cuda")
     dev = p.table.device
     n = min(n, w.seq_len)
     pos = [(0, t) for t in range(n)]
@@ -157,20 +165,20 @@ def oracle_sample(w, tokens: int, nthreads: int):
     return n, run
 
 
-def oracle_tokens_for(w, seconds: float, nthreads: int) -> int:
+def oracle_tokens_for(w, seconds: float, nthreads: int, p=None) -> int:
     """Sample size that takes about `seconds` of oracle time (calibrated)."""
-    n, run = oracle_sample(w, 32, nthreads)
+    n, run = oracle_sample(w, 32, nthreads, p)
     run()
     dt = run()
     return int(max(8, n / max(dt, 1e-6) * seconds))
 
 
-def cpu_baseline(w, budget_s: float):
+def cpu_baseline(w, budget_s: float, p=None):
     """The oracle on all host cores (the reported value) and on one core."""
     nthreads = os.cpu_count() or 1
-    n, run = oracle_sample(w, oracle_tokens_for(w, budget_s, nthreads), nthreads)
+    n, run = oracle_sample(w, oracle_tokens_for(w, budget_s, nthreads, p), nthreads, p)
     dt = run()
-    n1, run1 = oracle_sample(w, oracle_tokens_for(w, budget_s / 4, 1), 1)
+    n1, run1 = oracle_sample(w, oracle_tokens_for(w, budget_s / 4, 1, p), 1, p)
     dt1 = run1()
     return {"value": n / dt, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
             "single_thread_value": n1 / dt1,
@@ -242,6 +250,35 @@ def job_throughput(world, units_per_step_per_rank, steps, max_ms):
     return world * units_per_step_per_rank * steps / (max_ms / 1e3)
 
 
+def device_memory(w, p, ws, y):
+    """Device memory of one replica, GB: tables, weights, this step's inputs and
+    output, the forward workspace, and the library's static scratch (the array
+    behind engram_forward_no_alloc, held by every GPU that loads libengram.so
+    whether or not that entry point is called)."""
+    from hashed_gram_conditional_hash_b200 import _lib as L
+    nb = lambda t: t.numel() * t.element_size() if t is not None else 0
+    weights = sum(nb(t) for t in (p.w_value, p.w_key, p.norm_key, p.norm_query, p.conv_w, p.lookup))
+    return {"tables": round(nb(p.table) / 1e9, 3), "weights": round(weights / 1e9, 3),
+            "inputs_outputs": round((nb(p.ids) + nb(p.hidden) + nb(y)) / 1e9, 3),
+            "workspace": round(nb(ws) / 1e9, 3),
+            "static_scratch": round(L.NO_ALLOC_SCRATCH_BYTES / 1e9, 3)}
+
+
+class L2Flush:
+    """Between timed steps: write 256 MB (twice L2), then read another 256 MB
+    so that the written lines leave L2 now rather than during the next step's
+    first kernel (whose stage time would otherwise include that write-back)."""
+
+    def __init__(self, device):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+        self.src = torch.ones(32 << 20, dtype=torch.int64, device=device)
+        self.out = torch.empty((), dtype=torch.int64, device=device)
+
+    def __call__(self, i):
+        self.buf.fill_(i & 0xff)
+        torch.sum(self.src, dim=0, out=self.out)
+
+
 def run_ours(args, rank, world, device):
     from hashed_gram_conditional_hash_b200 import EngramLayer
     from hashed_gram_conditional_hash_b200 import _lib as L
@@ -270,7 +307,7 @@ def run_ours(args, rank, world, device):
         step_in = lambda i: (p.ids, p.hidden)
     ws = layer.workspace(Bq, Tq)
     y = torch.empty((Bq, Tq, w.hc_mult, w.hidden), dtype=w.torch_dtype, device=device)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     st = torch.zeros(1, dtype=torch.int32, device=device)
 
     def step(i):
@@ -279,7 +316,7 @@ def run_ours(args, rank, world, device):
 
     for i in range(args.warmup):
         step(i)
-        flush.fill_(i & 0xff)
+        flush(i)
     torch.cuda.synchronize()
     bits = L.engram_read_status(st)
     if bits:
@@ -311,7 +348,7 @@ def run_ours(args, rank, world, device):
         ev_step[i][0].record(stream)
         step(args.warmup + i)
         ev_step[i][1].record(stream)
-        flush.fill_(i & 0xff)
+        flush(i)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -321,7 +358,7 @@ def run_ours(args, rank, world, device):
         L.engram_set_stage_events(ev[i])
         step(args.warmup + K + i)
         L.engram_set_stage_events(None)
-        flush.fill_(i & 0xff)
+        flush(i)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -369,8 +406,9 @@ def run_ours(args, rank, world, device):
                    "orders": list(w.orders), "heads_per_order": w.heads_per_order,
                    "row_dim": w.row_dim, "hidden": w.hidden, "hc_mult": w.hc_mult,
                    "dilation": w.dil, "table_gb": round(W.table_bytes(w) / 1e9, 3),
-                   "l2": "flushed (256 MB write) between timed steps",
-                   "parallelism": "replicas x%d" % world, "projection_engine": engine},
+                   "l2": "flushed (256 MB write) and drained (256 MB read) between timed steps",
+                   "parallelism": "replicas x%d" % world, "projection_engine": engine,
+                   "device_memory_gb": device_memory(w, p, ws, y)},
         "roofline": {"bound": "tensor", "kernel": kname,
                      "achieved": proj_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": proj_tflops / tc_peak, "peak_kind": "%s bf16 %s" % (peak_kind, "sustained" if sustained else "burst"),
@@ -475,7 +513,7 @@ def run_offload(args, layer, p, w, device):
     ws = layer.workspace(B, T)
     y = torch.empty((B, T, w.hc_mult, w.hidden), dtype=w.torch_dtype, device=device)
     e = [hl.gather_ids(p.ids) for _ in range(2)]
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     comp = torch.cuda.current_stream()
     side = torch.cuda.Stream(device=device)
     ready, free = [torch.cuda.Event(), torch.cuda.Event()], [torch.cuda.Event(), torch.cuda.Event()]
@@ -486,14 +524,14 @@ def run_offload(args, layer, p, w, device):
     def timed(step):
         for i in range(3):
             step(i)
-            flush.fill_(i & 0xff)
+            flush(i)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(comp)
         side.wait_event(e0)
         for i in range(K):
             step(i)
-            flush.fill_(i & 0xff)
+            flush(i)
         comp.wait_stream(side)
         e1.record(comp)
         torch.cuda.synchronize()
@@ -503,7 +541,7 @@ def run_offload(args, layer, p, w, device):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(comp)
         for i in range(K):
-            flush.fill_(i & 0xff)
+            flush(i)
         e1.record(comp)
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / K
@@ -552,7 +590,9 @@ def run_offload(args, layer, p, w, device):
                     "layers' compute to hide the host-link transfer behind"}
 
 
-PEER_COPY_GBS = 770.0   # NVLink 5 peer copy rate measured on B200 HGX, per direction per GPU
+# Assumed NVLink 5 peer-copy rate per direction per GPU (a figure quoted for
+# B200 HGX nodes; no run of this bench has had two GPUs to measure it).
+PEER_COPY_GBS = 770.0
 
 
 def run_sharded(args, layer, p, w, device):
@@ -564,7 +604,7 @@ def run_sharded(args, layer, p, w, device):
     launch (timed as the N local rows of this batch served from shard 0, the
     largest, of total/R rows); place = engram_shard_place.  The two
     all-to-alls cannot run on one GPU: their per-rank bytes are reported with
-    the time they would take at the measured peer-copy rate, as an estimate."""
+    the time they would take at an assumed peer-copy rate, as an estimate."""
     from hashed_gram_conditional_hash_b200 import _lib as L
     R = args.sharded
     B, T = w.B, w.T
@@ -579,20 +619,20 @@ def run_sharded(args, layer, p, w, device):
     got = torch.empty((n, w.row_dim), dtype=p.table.dtype, device=device)
     e = torch.empty((B * T, w.nh * w.row_dim), dtype=p.table.dtype, device=device)
     L.engram_shard_route(layer.cfg, layer.weights, p.ids, R, counts, req_rows, req_pos, ws)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(device)
     K = max(3, min(args.steps, 200))
 
     def timed(step):
         for i in range(3):
             step()
-            flush.fill_(i & 0xff)
+            flush(i)
         torch.cuda.synchronize()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         for i in range(K):
             ev[i][0].record()
             step()
             ev[i][1].record()
-            flush.fill_(i & 0xff)
+            flush(i)
         torch.cuda.synchronize()
         return sorted(a.elapsed_time(b) * 1e3 for a, b in ev)[K // 2]     # median µs
 
@@ -613,20 +653,28 @@ def run_sharded(args, layer, p, w, device):
             "device_steps_us": t_steps,
             "exchange_bytes_per_rank_each_way": int(x_bytes),
             "exchange_us_estimated": x_bytes / (PEER_COPY_GBS * 1e3),
-            "note": "one GPU: device steps measured (medians, L2 flushed before each timed launch, so each "
-                    "part alone also pays the flush's write-back; device_steps_us is the three back to back "
-                    "after one flush); the two all-to-alls estimated from their bytes at %.0f GB/s per "
+            "note": "one GPU: device steps measured (medians, L2 flushed and drained before each timed "
+                    "launch; device_steps_us is the three back to back after one flush); the two "
+                    "all-to-alls estimated from their bytes at an assumed %.0f GB/s per "
                     "direction, not measured" % PEER_COPY_GBS}
 
 
+PROBE_OPS = {"write_v4": 0, "write_v8": 1, "write_v4_cs": 2, "write_bulk": 3, "read_v4": 4, "read_v8": 5,
+             "copy_v4": 6, "copy_v8": 7}
+
+
 def hbm_rates(device):
-    """Write-only, read-only and copy rates of HBM on 1 GiB buffers (torch fill,
-    sum and copy kernels; median of 20 launches by CUDA events): the read and
-    write sides of the roofline of kernels whose traffic is mostly one way."""
+    """HBM write-only, read-only and copy rates on 1 GiB buffers: this
+    library's probe kernels (16- and 32-byte stores and loads, evict-first
+    stores, bulk-copy-engine stores; libengram_probe.so) beside torch's fill,
+    sum and copy; median of 20 launches by CUDA events.  They are the write and
+    read sides of the roofline of kernels whose traffic is mostly one way."""
+    import ctypes
     n = 1 << 30
     a = torch.empty(n, dtype=torch.uint8, device=device)
     b = torch.empty_like(a)
     out = torch.empty((), dtype=torch.int64, device=device)
+    stream = torch.cuda.current_stream()
 
     def med_ms(fn):
         for _ in range(3):
@@ -641,11 +689,35 @@ def hbm_rates(device):
         return sorted(x.elapsed_time(y) for x, y in ev)[10]
 
     a.fill_(1)
-    t_w = med_ms(lambda: a.fill_(2))
-    t_r = med_ms(lambda: torch.sum(a.view(torch.int64), dim=0, out=out))
-    t_c = med_ms(lambda: b.copy_(a))
-    return {"write_only_gbs": n / t_w / 1e6, "read_only_gbs": n / t_r / 1e6, "copy_gbs": 2 * n / t_c / 1e6,
-            "bytes": n, "note": "torch fill_ / sum / copy_ on 1 GiB, median of 20 launches"}
+    res = {"bytes": n, "note": "1 GiB buffers, median of 20 launches; copy rates count bytes read + written"}
+    res["torch_fill_gbs"] = n / med_ms(lambda: a.fill_(2)) / 1e6
+    res["torch_sum_gbs"] = n / med_ms(lambda: torch.sum(a.view(torch.int64), dim=0, out=out)) / 1e6
+    res["torch_copy_gbs"] = 2 * n / med_ms(lambda: b.copy_(a)) / 1e6
+    from hashed_gram_conditional_hash_b200 import build as Bld
+    lib = ctypes.CDLL(Bld.PROBE_LIB)
+    lib.engram_probe_hbm.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                     ctypes.c_int, ctypes.c_void_p]
+    for name, op in PROBE_OPS.items():
+        best = None
+        for blocks_per_sm in (2, 4, 8):
+            blocks = blocks_per_sm * torch.cuda.get_device_properties(device).multi_processor_count
+            if name == "write_bulk":
+                blocks *= 4      # 32-thread blocks: one bulk-copy issuer each
+
+            def run():
+                rc = lib.engram_probe_hbm(op, b.data_ptr(), a.data_ptr(), n, blocks, stream.cuda_stream)
+                if rc != 0:
+                    raise RuntimeError("probe %s failed: %d" % (name, rc))
+            ms = med_ms(run)
+            rate = (2 if name.startswith("copy") else 1) * n / ms / 1e6
+            if best is None or rate > best[0]:
+                best = (rate, blocks)
+        res[name + "_gbs"] = best[0]
+        res[name + "_blocks"] = best[1]
+    res["write_only_gbs"] = max(res[k + "_gbs"] for k in ("write_v4", "write_v8", "write_v4_cs", "write_bulk"))
+    res["read_only_gbs"] = max(res["read_v4_gbs"], res["read_v8_gbs"])
+    res["copy_gbs"] = max(res["copy_v4_gbs"], res["copy_v8_gbs"])
+    return res
 
 
 def run_reference(args):
@@ -655,7 +727,10 @@ def run_reference(args):
     w = W.CONFIGS[args.config]
     nthreads = os.cpu_count() or 1
     per_step = min(args.ref_step_s, 120.0 / max(1, args.steps + args.warmup))
-    n, run = oracle_sample(w, oracle_tokens_for(w, per_step, nthreads), nthreads)
+    # tables above 1 GiB are drawn on the GPU (plumbing only: the oracle runs
+    # on the host cores and receives the table rows its sample needs)
+    p = W.make_params(w, "cuda") if W.gen_device_for(w, "cuda") != "cpu" else None
+    n, run = oracle_sample(w, oracle_tokens_for(w, per_step, nthreads, p), nthreads, p)
     for _ in range(args.warmup):
         run()
     tot = 0.0
@@ -683,7 +758,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="model_bf16")
+    ap.add_argument("--config", default="hbm_table_bf16")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--ref-step-s", type=float, default=3.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -723,10 +798,14 @@ def main():
             res["hbm_rates"] = hbm_rates(device)
         if args.sharded and not w.decode_calls:
             res["sharded"] = run_sharded(args, layer, p, w, device)
+        from hashed_gram_conditional_hash_b200 import workloads as W
+        # device-drawn tables are kept for the oracle's sample (it fetches its rows)
+        keep = p if W.gen_device_for(w, device) != "cpu" else None
         del layer, p
         torch.cuda.empty_cache()
         if rank == 0 and not args.no_cpu_baseline and world == 1:
-            res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget_s)
+            res["cpu_baseline"] = cpu_baseline(w, args.cpu_budget_s, keep)
+        del keep
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
