@@ -3,7 +3,8 @@ token per engram_forward call for 256 calls, carrying the id ring and the
 V/gate rings in an engram_state.  Checked against the oracle's prefill over the
 same 256-token sequences at sampled positions, and against this library's own
 prefill over T = 256 (same kernels, so agreement is to rounding of identical
-operations), plus chunked prefill with the state."""
+operations), plus chunked prefill with the state, whose concatenated output is
+checked against the oracle's prefill over the whole sequence."""
 import numpy as np
 import pytest
 import torch
@@ -12,7 +13,7 @@ from hashed_gram_conditional_hash_b200 import EngramLayer
 from hashed_gram_conditional_hash_b200 import _lib as L
 from hashed_gram_conditional_hash_b200 import workloads as W
 
-from gpu_helpers import TOL, device_params, oracle_at, rel_err, sample_positions
+from gpu_helpers import TOL, device_params, oracle_at, oracle_forward_full, rel_err, sample_positions
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -73,6 +74,9 @@ def test_chunked_prefill_with_state(chunks):
     err = (y.double() - y_full.double()).abs().max().item()
     assert err <= 1e-2 * y_full.double().abs().max().item()
     assert torch.all(state.pos == t0)
+    # the chunks together are the oracle's prefill over the whole sequence
+    ref = oracle_forward_full(p)
+    assert rel_err(y.double().cpu().numpy(), ref["Y"]) <= TOL[w.dtype]
 
 
 def test_streaming_with_raw_ids_keeps_compressed_ids_in_the_ring():
@@ -91,5 +95,6 @@ def test_streaming_with_raw_ids_keeps_compressed_ids_in_the_ring():
     y = torch.cat(outs, 1)
     err = (y.double() - y_full.double()).abs().max().item()
     assert err <= 1e-2 * y_full.double().abs().max().item()
+    assert rel_err(y.double().cpu().numpy(), oracle_forward_full(p)["Y"]) <= TOL[w.dtype]
     assert torch.equal(state.id_ring, p.lookup[p.ids[:, -(w.max_n - 1):]])
     assert torch.all(state.pos == w.T)

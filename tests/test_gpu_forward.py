@@ -73,11 +73,16 @@ def test_forward_tiny_f32_full():
     assert err <= TOL["f32"], err
 
 
-@pytest.mark.parametrize("name", ["model_bf16", "large_table_bf16", "hbm_table_bf16"])
+@pytest.mark.parametrize("name", ["model_bf16", "model_bf16_norm_w", "large_table_bf16", "hbm_table_bf16"])
 def test_forward_full_size_sampled(name):
     # the bench's launch configuration at full size: both tensor-core engines
-    # against the oracle at the sequence edges plus 4096 random positions
-    w = W.CONFIGS[name]
+    # against the oracle at the sequence edges plus 4096 random positions;
+    # "_norm_w": RMSNorm weights 1 + N(0, 0.1^2) instead of exactly 1, so the
+    # weight products of the key epilogue are exercised at full size
+    if name.endswith("_norm_w"):
+        w = W.CONFIGS[name[: -len("_norm_w")]].replace(norm_w_std=0.1)
+    else:
+        w = W.CONFIGS[name]
     p = device_params(w)
     pos = sample_positions(w.B, w.T, w.dil, 4096, seed=11)
     Yref, _, _, _ = oracle_at(p, pos)
@@ -116,6 +121,19 @@ def test_forward_zero_conv_is_gated_value():
     y = _run(p, conv_w=zero)
     ref = oracle_forward_full(p, conv_w=zero)
     assert rel_err(y.double().cpu().numpy(), ref["g"][..., None] * ref["V"][:, :, None, :]) <= TOL["bf16"]
+
+
+def test_forward_branch_with_zero_hidden_gates_one_half():
+    # a branch whose hidden state is zero has s = 0, so g = 1/2 exactly
+    # (formulas page §2.2 step 2) and its Y is the conv of V/2
+    w = W.small_workload(B=2, T=100, hidden=512, hc_mult=4)
+    p = device_params(w)
+    p.hidden[:, :, 2] = 0
+    ref = oracle_forward_full(p)
+    assert np.all(ref["s"][:, :, 2] == 0.0) and np.all(ref["g"][:, :, 2] == 0.5)
+    for engine in ("auto", "simt"):
+        y = _run(p, engine)
+        assert rel_err(y.double().cpu().numpy(), ref["Y"]) <= TOL["bf16"], engine
 
 
 def test_forward_split_value_tail_tiles():

@@ -86,6 +86,16 @@ def test_pageable_host_table_is_refused_without_launch():
     assert L.engram_launch_count() == before
 
 
+def _oracle_rows(p, x, hist=None):
+    """Each row of e as the oracle gives it: the table row at the oracle's
+    index (its own multipliers and primes), for a table on the device or in
+    pinned host memory."""
+    w = p.w
+    idx = O.ngram_hash(x, w.orders, w.heads_per_order, p.mult, p.primes, w.pad_id, hist=hist)
+    rows = torch.from_numpy((idx + np.asarray(p.offsets)[None, None, :]).reshape(-1))
+    return p.table[rows.to(p.table.device)].reshape(x.shape[0] * x.shape[1], w.nh * w.row_dim).cpu()
+
+
 def test_gather_ids_layers_equals_per_layer_gathers():
     # two Engram layers of one model (the pages' layers 2 and 6): own
     # multipliers and tables, the same ids; one host-resident table
@@ -101,8 +111,12 @@ def test_gather_ids_layers_equals_per_layer_gathers():
          for _ in layers]
     L.engram_gather_ids_layers(layers[0].cfg, [l.weights for l in layers], ids, e, dev_status=st)
     assert L.engram_read_status(st) == 0
-    for layer, e_l in zip(layers, e):
+    x = oracle_ids(ps[0])
+    for p_l, layer, e_l in zip(ps, layers, e):
         assert torch.equal(e_l, layer.gather_ids(ids))
+        # every layer's rows, bit for bit, from the oracle's hash with that
+        # layer's multipliers and primes and that layer's table
+        assert torch.equal(e_l.cpu(), _oracle_rows(p_l, x))
     # and the rows reach each layer's own forward
     y0 = layers[0].forward_gathered(e[0], ps[0].hidden)
     assert torch.equal(y0, layers[0].forward(ids, ps[0].hidden))
@@ -120,6 +134,9 @@ def test_gather_ids_layers_with_history_continues_sequences():
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
     L.engram_gather_ids_layers(layers[0].cfg, [l.weights for l in layers], tail, e, history=hist, dev_status=st)
     assert L.engram_read_status(st) == 0
-    for layer, e_l in zip(layers, e):
+    x = ids.cpu().numpy()
+    for p_l, layer, e_l in zip(ps, layers, e):
         full = layer.gather_ids(ids)
         assert torch.equal(e_l.view(base.B, -1, E), full.view(base.B, base.T, E)[:, 20:])
+        # the oracle's hash of the tail with the same history
+        assert torch.equal(e_l.cpu(), _oracle_rows(p_l, x[:, 20:], hist=x[:, 17:20]))

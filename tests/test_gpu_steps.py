@@ -145,6 +145,36 @@ def test_gate_fuse_parity(dtype, H, hc, M):
     assert np.max(np.abs(gates.double().cpu().numpy() - gref)[mask]) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("engine", ["auto", "simt"])
+def test_gate_is_one_half_exactly_when_a_branch_sees_zero_hidden(engine):
+    # formulas page §2.2 step 2 with sign(0) = 0: a zero query gives s = 0,
+    # hence g = sigmoid(0) = 1/2 exactly, and u = V/2 for that branch
+    w = W.small_workload(hidden=512, hc_mult=4)
+    p = device_params(w)
+    M = 300
+    g = torch.Generator(device="cpu").manual_seed(13)
+    e = (0.02 * torch.randn(M, w.E, generator=g)).to(w.torch_dtype).to(DEV)
+    hid = torch.randn(M, w.hc_mult, w.hidden, generator=g).to(w.torch_dtype)
+    hid[:, 1] = 0
+    hid = hid.to(DEV)
+    u = torch.empty((M, w.hc_mult, w.hidden), dtype=w.torch_dtype, device=DEV)
+    gates = torch.empty((M, w.hc_mult), dtype=torch.float32, device=DEV)
+    L.engram_set_debug(L.DEBUG_FORCE_SIMT if engine == "simt" else 0)
+    try:
+        L.engram_gate_fuse(_cfg(w), e, p.w_value, p.w_key, p.norm_key, p.norm_query, hid, u, gates)
+        torch.cuda.synchronize()
+    finally:
+        L.engram_set_debug(0)
+    assert torch.all(gates[:, 1] == 0.5)
+    V, s, gref = O.tokens_gate(O.widen(*O.storage(e)), w.hidden, w.hc_mult, p.w_value.cpu(), p.w_key.cpu(),
+                               p.norm_key.cpu(), p.norm_query.cpu(), hid.cpu(), w.rms_eps, w.gate_eps)
+    assert np.all(s[:, 1] == 0.0) and np.all(gref[:, 1] == 0.5)
+    assert rel_err(u.double().cpu().numpy(), gref[:, :, None] * V[:, None, :]) <= TOL["bf16"]
+    # the other branches keep their gates (masking the sign-ambiguous |s| < 1e-5)
+    mask = np.abs(s) >= 1e-5
+    assert np.max(np.abs(gates.double().cpu().numpy() - gref)[mask]) <= TOL["bf16"]
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_short_conv_parity_and_state(dtype):
     w = W.small_workload(dtype=dtype, hidden=128, hc_mult=2)
