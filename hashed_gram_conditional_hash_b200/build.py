@@ -3,7 +3,8 @@
 Each .cu file under csrc/ is compiled to an object (rebuilt when it or a
 header is newer) and the objects are linked into
 hashed_gram_conditional_hash_b200/libengram.so with the CUDA runtime linked
-statically.
+statically.  The benchmark's HBM rate probes (probe/) build into a separate
+libengram_probe.so.
 """
 from __future__ import annotations
 
@@ -19,6 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libengram.so")
 INCLUDE = os.path.join(ROOT, "include")
+PROBE = os.path.join(PKG, "probe")
+PROBE_LIB = os.path.join(PKG, "libengram_probe.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
@@ -61,7 +64,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
         cmd = [nvcc()] + ARCH + ["-shared", "-o", tmp] + objs + ["-cudart", "static"]
         subprocess.check_call(cmd)
         os.replace(tmp, LIB)
+    build_probe(force)
     return LIB
+
+
+def build_probe(force: bool = False) -> str:
+    """libengram_probe.so: the benchmark's HBM rate probes (not the pass)."""
+    src = os.path.join(PROBE, "hbm_probe.cu")
+    if force or not os.path.exists(PROBE_LIB) or os.path.getmtime(PROBE_LIB) < os.path.getmtime(src):
+        tmp = PROBE_LIB + ".tmp%d" % os.getpid()
+        cmd = [nvcc()] + ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
+                                  src, "-o", tmp, "-cudart", "static"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, PROBE_LIB)
+    return PROBE_LIB
 
 
 if __name__ == "__main__":

@@ -1,0 +1,146 @@
+// HBM rate probes for the benchmark (not part of the Engram pass): how fast
+// this GPU writes, reads and copies a large buffer with the store and load
+// forms the pass's kernels can use.  They set the write-side and read-side
+// ceilings against which kernels whose traffic is mostly one way (the conv
+// writes hc times the bytes it reads) are judged, instead of a library
+// kernel's rate.
+//
+// ops (bytes a multiple of 32, pointers 32-byte aligned):
+//   0 write, 16-byte st.global.v4         1 write, 32-byte st.global.v8
+//   2 write, 16-byte st.global.cs (evict-first)
+//   3 write, cp.async.bulk from a 32 KB shared tile (the bulk-copy engine)
+//   4 read, 16-byte ld.global.nc          5 read, 32-byte ld.global.nc.v8
+//   6 copy, 16-byte                        7 copy, 32-byte
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace {
+
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ void st16(void* p, uint32_t v) {
+  asm volatile("st.global.v4.b32 [%0], {%1, %1, %1, %1};" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st16cs(void* p, uint32_t v) {
+  asm volatile("st.global.cs.v4.b32 [%0], {%1, %1, %1, %1};" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st32(void* p, uint32_t v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1};" ::"l"(p), "r"(v) : "memory");
+}
+
+// Grid-stride over units of U bytes, kUnroll independent accesses per step.
+template <int OP, int U>
+__global__ void __launch_bounds__(256) rw_kernel(char* dst, const char* src, int64_t n_units, uint32_t* sink) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint32_t acc = 0;
+  const uint32_t val = static_cast<uint32_t>(tid) | 1u;
+  for (int64_t base = tid; base < n_units; base += stride * kUnroll) {
+    if (OP == 0 || OP == 1 || OP == 2) {
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * stride;
+        if (i < n_units) {
+          if (OP == 1) st32(dst + i * U, val);
+          else if (OP == 2) st16cs(dst + i * U, val);
+          else st16(dst + i * U, val);
+        }
+      }
+    } else {
+      uint32_t r[kUnroll][8];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * stride;
+        if (i < n_units) {
+          const char* p = src + i * U;
+          if (U == 32)
+            asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                         : "=r"(r[u][0]), "=r"(r[u][1]), "=r"(r[u][2]), "=r"(r[u][3]), "=r"(r[u][4]),
+                           "=r"(r[u][5]), "=r"(r[u][6]), "=r"(r[u][7])
+                         : "l"(p));
+          else
+            asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(r[u][0]), "=r"(r[u][1]), "=r"(r[u][2]), "=r"(r[u][3])
+                         : "l"(p));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t i = base + u * stride;
+        if (i >= n_units) continue;
+        if (OP == 4 || OP == 5) {
+#pragma unroll
+          for (int k = 0; k < U / 4; ++k) acc ^= r[u][k];
+        } else if (U == 32) {
+          asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst + i * U), "r"(r[u][0]),
+                       "r"(r[u][1]), "r"(r[u][2]), "r"(r[u][3]), "r"(r[u][4]), "r"(r[u][5]), "r"(r[u][6]),
+                       "r"(r[u][7])
+                       : "memory");
+        } else {
+          asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(dst + i * U), "r"(r[u][0]), "r"(r[u][1]),
+                       "r"(r[u][2]), "r"(r[u][3])
+                       : "memory");
+        }
+      }
+    }
+  }
+  if ((OP == 4 || OP == 5) && acc == 0x9e3779b9u) sink[0] = acc;  // keeps the loads live
+}
+
+// Bulk-copy engine writes: each block owns contiguous 32 KB chunks (grid-
+// stride), copied from one shared tile that is never modified, so the
+// copies need no wait between them; all complete before the block exits.
+constexpr int kChunk = 32 * 1024;
+__global__ void __launch_bounds__(32) bulk_write_kernel(char* dst, int64_t n_chunks) {
+  extern __shared__ __align__(128) uint4 tile[];
+  for (int i = threadIdx.x; i < kChunk / 16; i += 32) tile[i] = make_uint4(i, i, i, i);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(tile));
+    for (int64_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
+      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst + c * kChunk), "r"(s),
+                   "r"(kChunk)
+                   : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+  __syncwarp();
+}
+
+}  // namespace
+
+// Runs op once on the stream; blocks = grid size (<= 0: 4 per SM).  Returns a
+// cudaError_t.
+extern "C" int engram_probe_hbm(int op, void* dst, const void* src, size_t bytes, int blocks, void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (bytes % 32 != 0 || (reinterpret_cast<uintptr_t>(dst) & 31u) != 0 ||
+      (reinterpret_cast<uintptr_t>(src) & 31u) != 0)
+    return static_cast<int>(cudaErrorInvalidValue);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (blocks <= 0) blocks = 4 * sms;
+  char* d = static_cast<char*>(dst);
+  const char* r = static_cast<const char*>(src);
+  uint32_t* sink = static_cast<uint32_t*>(dst);
+  const int64_t n16 = static_cast<int64_t>(bytes / 16), n32 = static_cast<int64_t>(bytes / 32);
+  switch (op) {
+    case 0: rw_kernel<0, 16><<<blocks, 256, 0, s>>>(d, r, n16, sink); break;
+    case 1: rw_kernel<1, 32><<<blocks, 256, 0, s>>>(d, r, n32, sink); break;
+    case 2: rw_kernel<2, 16><<<blocks, 256, 0, s>>>(d, r, n16, sink); break;
+    case 3: {
+      if (bytes % kChunk != 0) return static_cast<int>(cudaErrorInvalidValue);
+      cudaFuncSetAttribute(bulk_write_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kChunk);
+      bulk_write_kernel<<<blocks, 32, kChunk, s>>>(d, static_cast<int64_t>(bytes / kChunk));
+      break;
+    }
+    case 4: rw_kernel<4, 16><<<blocks, 256, 0, s>>>(d, r, n16, sink); break;
+    case 5: rw_kernel<5, 32><<<blocks, 256, 0, s>>>(d, r, n32, sink); break;
+    case 6: rw_kernel<6, 16><<<blocks, 256, 0, s>>>(d, r, n16, sink); break;
+    case 7: rw_kernel<7, 32><<<blocks, 256, 0, s>>>(d, r, n32, sink); break;
+    default: return static_cast<int>(cudaErrorInvalidValue);
+  }
+  return static_cast<int>(cudaGetLastError());
+}
