@@ -196,6 +196,143 @@ __device__ __forceinline__ void hash_gather_body(const HashGatherParams& g) {
   }
 }
 
+// ---- the 128-byte-row form: 32 rows of e per warp, one pass of hashing
+//
+// Rows of e are head-minor (row q = m*nh + h), so a warp's 32 consecutive rows
+// cover at most floor((nh - 1 + 31) / nh) + 1 tokens.  Lane j loads the id at
+// flat position m_first - n_hist + j once (one coalesced load for the warp);
+// every lane then builds its own row's n-gram window from those registers by
+// shuffles (positions before its sequence's start come from the history or
+// pad_id), forms the mix of its order and reduces it by its head's prime.
+// The per-head constants sit in shared memory: indexing the kernel's
+// parameter space by a per-lane head would serialise across the warp.  The
+// rows then move as 32-byte pieces (four per 128-byte row, four per lane per
+// chunk), every load issued before the first store.  Ids are below 2^32 and
+// table rows below 2^31 (both checked on the host), so the shuffles move
+// 32-bit values.  NC chunks of 32 rows per warp are hashed first and copied
+// together (NC = 1 in use: a warp keeps 4 KB of row reads in flight; two
+// chunks per warp, fewer and longer warps, measured slower on the HBM-scale
+// table, 158 vs 106 us).
+struct HeadConst {
+  uint64_t prime, mu;       // modulus and its Barrett constant
+  int32_t row_off, order;   // first table row of the head, n of its order
+};
+
+__device__ __forceinline__ void ld_row32(const char* p, uint4& a, uint4& b) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+               : "l"(p));
+}
+__device__ __forceinline__ void st_row32(char* p, const uint4& a, const uint4& b) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+               "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
+
+// Id at position t < 0 of sequence b: the history (most recent last), else pad.
+__device__ __forceinline__ uint64_t id_before_start(const HashParams& p, int b, int t) {
+  if (p.history != nullptr && -t <= p.n_hist) {
+    int64_t hv = __ldg(p.history + static_cast<int64_t>(b) * p.n_hist + p.n_hist + t);
+    if (hv < 0 || hv >= p.vocab) {
+      set_status(p.status, ENGRAM_STATUS_ID_RANGE);
+      hv = p.pad_id;
+    }
+    return static_cast<uint64_t>(hv);
+  }
+  return static_cast<uint64_t>(p.pad_id);
+}
+
+template <int NC>
+__device__ __forceinline__ void hash_gather_w32_body(const HashGatherParams& g, const HeadConst* hcs) {
+  const HashParams& p = g.h;
+  const int lane = threadIdx.x & 31;
+  const int gtid = static_cast<int>(blockIdx.x * blockDim.x + threadIdx.x);
+  if (g.wprod != nullptr)   // the RMSNorm weight products of the score, for the projection
+    for (int i = gtid; i < g.n_w; i += static_cast<int>(gridDim.x * blockDim.x))
+      g.wprod[i] = bf16_to_f32(__ldg(g.nk + i)) * bf16_to_f32(__ldg(g.nq + i));
+  const int M = p.B * p.T;
+  const int total = M * p.nh;                       // < 2^31 (checked by the launcher)
+  const int qw = (gtid >> 5) * (32 * NC);           // first row of the warp
+  if (qw >= total) return;
+  int32_t row[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const int q0 = qw + 32 * c;
+    row[c] = 0;
+    if (q0 >= total) continue;                      // (warp-uniform)
+    const int m_first = static_cast<int>(fast_div(static_cast<uint32_t>(q0), g.div_nh));
+    const int wpos = m_first - p.n_hist + lane;     // this lane's id of the window
+    uint32_t xw = static_cast<uint32_t>(p.pad_id);
+    if (wpos >= 0 && wpos < M) xw = static_cast<uint32_t>(load_id(p, __ldg(p.ids + wpos)));
+    const int q = min(q0 + lane, total - 1);
+    const int m = static_cast<int>(fast_div(static_cast<uint32_t>(q), g.div_nh));
+    const int h = q - m * p.nh;
+    const HeadConst hc = hcs[h];
+    const int b = static_cast<int>(fast_div(static_cast<uint32_t>(m), g.div_T));
+    const int t = m - b * p.T;
+    const int src = m - m_first + p.n_hist;         // lane holding x[m]
+    uint64_t mix = 0;
+    for (int k = 0; k <= p.n_hist; ++k) {           // warp-uniform bound
+      const uint32_t v = __shfl_sync(0xffffffffu, xw, (src - k) & 31);
+      if (k < hc.order) {
+        const uint64_t tok = t >= k ? static_cast<uint64_t>(v) : id_before_start(p, b, t - k);
+        const uint64_t prod = tok * p.mult[k];
+        mix = k == 0 ? prod : (mix ^ prod);
+      }
+    }
+    row[c] = hc.row_off + static_cast<int32_t>(barrett_mod(mix, hc.prime, hc.mu));
+  }
+  // piece i of a chunk = row i / 4, 32-byte column i % 4
+  const char* tab = static_cast<const char*>(g.table);
+  uint4 va[NC][4], vb[NC][4];
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = u * 32 + lane;
+      const int r = i >> 2;
+      const int32_t srow = __shfl_sync(0xffffffffu, row[c], r);
+      if (qw + 32 * c + r < total)
+        ld_row32(tab + static_cast<int64_t>(srow) * 128 + (i & 3) * 32, va[c][u], vb[c][u]);
+    }
+  char* out = static_cast<char*>(g.e) + static_cast<int64_t>(qw) * 128;
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = u * 32 + lane;
+      if (qw + 32 * c + (i >> 2) < total) st_row32(out + (c * 128 + i) * 32, va[c][u], vb[c][u]);
+    }
+}
+
+__device__ __forceinline__ void load_head_consts(const HashParams& p, HeadConst* hcs) {
+  for (int i = static_cast<int>(threadIdx.x); i < p.nh; i += static_cast<int>(blockDim.x)) {
+    HeadConst c;
+    c.prime = p.prime[i];
+    c.mu = p.barrett[i];
+    c.row_off = static_cast<int32_t>(p.row_off[i]);
+    c.order = p.orders[i / p.J];
+    hcs[i] = c;
+  }
+  __syncthreads();
+}
+
+template <int NC>
+__global__ void __launch_bounds__(256) hash_gather_w32_kernel(const __grid_constant__ HashGatherParams g) {
+  __shared__ HeadConst hcs[ENGRAM_MAX_HEADS];
+  load_head_consts(g.h, hcs);   // kernel parameters only: before the wait
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  hash_gather_w32_body<NC>(g, hcs);
+}
+
+template <int NC>
+__global__ void __launch_bounds__(256) hash_gather_w32_layers_kernel(const __grid_constant__ HashGatherLayers g) {
+  __shared__ HeadConst hcs[ENGRAM_MAX_HEADS];
+  load_head_consts(g.layer[blockIdx.y].h, hcs);
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  hash_gather_w32_body<NC>(g.layer[blockIdx.y], hcs);
+}
+
 template <int CH, int ROWS, bool HOSTMEM>
 __global__ void __launch_bounds__(256) hash_gather_kernel(const __grid_constant__ HashGatherParams g) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
@@ -342,6 +479,14 @@ __global__ void compress_kernel(const int64_t* __restrict__ raw, int64_t n,
 
 }  // namespace
 
+// The 32-row form: 128-byte rows of a device table, table and e 32-byte
+// aligned (for the 32-byte accesses), at least two heads (so the ids of a
+// warp's tokens and their n-gram windows fit one register per lane).
+bool w32_form(const HashGatherParams& g) {
+  return g.row_bytes == 128 && !g.table_host && g.h.nh >= 2 &&
+         ((reinterpret_cast<uintptr_t>(g.table) | reinterpret_cast<uintptr_t>(g.e)) & 31u) == 0;
+}
+
 cudaError_t launch_hash(const HashParams& p, cudaStream_t s) {
   if (p.B > 0 && p.T > 0) {
     dim3 grid((p.T + 255) / 256, p.B);
@@ -362,7 +507,10 @@ cudaError_t launch_hash_gather(const HashGatherParams& g0, cudaStream_t s) {
   if (total > 0) {
     constexpr int kRows = 16;                    // rows per warp for 128-byte rows
     if (total * (32 / kRows) + 256 > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit ids in the kernel
-    if (g.row_bytes == 128) {
+    if (w32_form(g)) {
+      const int64_t blocks = (total + 255) / 256;
+      launch_k(hash_gather_w32_kernel<1>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
+    } else if (g.row_bytes == 128) {
       const int64_t blocks = (total + 8 * kRows - 1) / (8 * kRows);
       if (g.table_host)
         launch_k(hash_gather_kernel<8, kRows, true>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
@@ -400,7 +548,12 @@ cudaError_t launch_hash_gather_layers(const HashGatherLayers& g0, cudaStream_t s
   constexpr int kRows = 16;
   if (total * (32 / kRows) + 256 > INT32_MAX) return cudaErrorInvalidValue;
   const unsigned layers = static_cast<unsigned>(g.n_layers);
-  if (g.layer[0].row_bytes == 128) {
+  bool w32 = true;
+  for (int l = 0; l < g.n_layers; ++l) w32 = w32 && w32_form(g.layer[l]);
+  if (w32) {
+    const dim3 grid(static_cast<unsigned>((total + 255) / 256), layers);
+    launch_k(hash_gather_w32_layers_kernel<1>, grid, dim3(256), 0, s, g);
+  } else if (g.layer[0].row_bytes == 128) {
     const dim3 grid(static_cast<unsigned>((total + 8 * kRows - 1) / (8 * kRows)), layers);
     if (host) launch_k(hash_gather_layers_kernel<8, kRows, true>, grid, dim3(256), 0, s, g);
     else launch_k(hash_gather_layers_kernel<8, kRows, false>, grid, dim3(256), 0, s, g);

@@ -96,6 +96,43 @@ def _oracle_rows(p, x, hist=None):
     return p.table[rows.to(p.table.device)].reshape(x.shape[0] * x.shape[1], w.nh * w.row_dim).cpu()
 
 
+GATHER_SHAPES = [
+    dict(B=3, T=5, orders=(2, 3), heads_per_order=1),              # 2 heads: a warp spans many short sequences
+    dict(B=4, T=7, orders=(2, 3, 4), heads_per_order=1),           # 3 heads (odd), rows cross tokens mid-warp
+    dict(B=2, T=33, orders=(2,), heads_per_order=1),               # 1 head: the 16-row form
+    dict(B=2, T=19, orders=(1, 2, 3, 4, 5, 6, 7, 8), heads_per_order=8, vocab=3000),  # 64 heads, order 8
+    dict(B=5, T=61, orders=(2, 3, 4), heads_per_order=5),          # 15 heads
+    dict(B=1, T=1),                                                # a single token
+]
+
+
+@pytest.mark.parametrize("kw", GATHER_SHAPES, ids=[str(i) for i in range(len(GATHER_SHAPES))])
+@pytest.mark.parametrize("with_history", [False, True])
+def test_gather_ids_bit_exact_against_oracle(kw, with_history):
+    # the hash + gather kernel's rows, bit for bit, over shapes that put the
+    # edges of sequences and tokens at every place inside a warp's rows
+    w = W.small_workload(prime_base=1009, **kw)
+    p = device_params(w)
+    layer = _layer(p)
+    x = oracle_ids(p)
+    hist = None
+    if with_history:
+        g = np.random.default_rng(5)
+        hist = torch.from_numpy(g.integers(0, w.vocab, size=(w.B, w.max_n - 1))).to(DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    e = layer.gather_ids(p.ids, history=hist, dev_status=st)
+    assert L.engram_read_status(st) == 0
+    expect = _oracle_rows(p, x, hist=None if hist is None else hist.cpu().numpy())
+    assert torch.equal(e.cpu(), expect)
+    # e 16 bytes off a 32-byte boundary takes the 16-byte form: same rows
+    buf = torch.empty(e.numel() * e.element_size() + 64, dtype=torch.uint8, device=DEV)
+    off = (16 - buf.data_ptr() % 32) % 32
+    e16 = buf[off: off + e.numel() * e.element_size()].view(e.dtype).view(e.shape)
+    assert e16.data_ptr() % 32 == 16
+    layer.gather_ids(p.ids, e=e16, history=hist)
+    assert torch.equal(e16.cpu(), expect)
+
+
 def test_gather_ids_layers_equals_per_layer_gathers():
     # two Engram layers of one model (the pages' layers 2 and 6): own
     # multipliers and tables, the same ids; one host-resident table
