@@ -288,6 +288,7 @@ def run_ours(args, rank, world, device):
     if w.decode_calls and args.decode_calls:
         w = w.replace(decode_calls=args.decode_calls)
     peaks, peak_kind = load_peaks()
+    L.engram_set_overlap_chunks(args.overlap_chunks)
     p = W.make_params(w, device)
     layer = EngramLayer.from_params(p)
     engine = "tcgen05" if L.engram_projection_engine(layer.cfg) == L.ENGINE_TCGEN05 else "simt"
@@ -408,7 +409,9 @@ def run_ours(args, rank, world, device):
                    "dilation": w.dil, "table_gb": round(W.table_bytes(w) / 1e9, 3),
                    "l2": "flushed (256 MB write) and drained (256 MB read) between timed steps",
                    "parallelism": "replicas x%d" % world, "projection_engine": engine,
-                   "device_memory_gb": device_memory(w, p, ws, y)},
+                   "device_memory_gb": device_memory(w, p, ws, y),
+                   "overlap_chunks": 1 if decode else min(w.B, 8, max(1, args.overlap_chunks or
+                                                                        int(os.environ.get("ENGRAM_OVERLAP_CHUNKS", "1"))))},
         "roofline": {"bound": "tensor", "kernel": kname,
                      "achieved": proj_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": proj_tflops / tc_peak, "peak_kind": "%s bf16 %s" % (peak_kind, "sustained" if sustained else "burst"),
@@ -763,6 +766,9 @@ def main():
     ap.add_argument("--ref-step-s", type=float, default=3.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--overlap-chunks", type=int, default=0,
+                    help="prefill in this many sequence chunks whose gate and conv overlap the next "
+                         "chunk's projection (0: the library default)")
     ap.add_argument("--decode-calls", type=int, default=0,
                     help="decode workload: number of distinct calls drawn (default: all 256)")
     ap.add_argument("--offload", action="store_true",

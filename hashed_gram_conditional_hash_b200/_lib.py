@@ -23,6 +23,7 @@ MAX_ORDERS = 8
 ENGRAM_F32, ENGRAM_BF16 = 0, 1
 STATUS_ID_RANGE, STATUS_ROW_RANGE, STATUS_TIMEOUT = 0x1, 0x2, 0x4
 DEBUG_FORCE_TIMEOUT, DEBUG_FORCE_SIMT, DEBUG_FUSED_GATHER, DEBUG_TC_SINGLE_CTA, DEBUG_NO_PDL = 0x1, 0x2, 0x4, 0x8, 0x10
+DEBUG_NO_OVERLAP = 0x20
 STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_CUDA",
                 4: "ERR_TIMEOUT", 5: "ERR_ID_RANGE"}
 
@@ -80,6 +81,7 @@ def lib() -> C.CDLL:
             "engram_last_error": (sz, [C.c_char_p, sz]),
             "engram_read_status": (C.c_int, [P, P, P]),
             "engram_set_debug": (None, [C.c_uint32]),
+            "engram_set_overlap_chunks": (None, [C.c_int32]),
             "engram_projection_engine": (i32, [cfg]),
             "engram_launch_count": (C.c_uint64, []),
             "engram_set_stage_events": (None, [C.POINTER(EngramStageEvents)]),
@@ -185,6 +187,12 @@ def engram_launch_count() -> int:
 
 def engram_set_debug(flags: int) -> None:
     lib().engram_set_debug(flags)
+
+
+def engram_set_overlap_chunks(chunks: int) -> None:
+    """Sequence chunks of a prefill whose gate and conv overlap the next
+    chunk's projection (<= 0: the default)."""
+    lib().engram_set_overlap_chunks(chunks)
 
 
 def engram_set_stage_events(events: Optional[dict]) -> None:

@@ -4,7 +4,10 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <stdlib.h>
+
 #include <atomic>
+#include <mutex>
 
 #include "engram_internal.cuh"
 
@@ -266,6 +269,136 @@ engram_status prepare_gather(const engram_config* cfg, const engram_weights* wts
   return ENGRAM_OK;
 }
 
+// ---- the pass in sequence chunks on two streams
+//
+// For a prefill on the CTA-pair projection, the batch may run as C chunks of
+// whole sequences: each chunk's projection on a high-priority internal
+// stream, back to back, and each chunk's gate and conv on a low-priority
+// internal stream as soon as its projection is done, so chunk i's gate and
+// conv run while chunk i + 1 is projected.  The projection kernel holds one
+// CTA per SM but leaves room for one block of the slim conv (no shared
+// memory, <= 88 registers at 128 threads) and of the gate; the high priority
+// puts the next projection's CTAs on the SMs first.  The last chunk's conv
+// has the GPU to itself and takes the tile form.  Chunks are whole
+// sequences, so no conv window crosses a chunk boundary.
+struct OverlapStreams {
+  cudaStream_t hi = nullptr, lo = nullptr;
+  cudaEvent_t fork = nullptr, proj = nullptr, hi_done = nullptr, lo_done = nullptr;
+  bool ok = false;
+};
+std::mutex g_overlap_mu;     // one caller at a time enqueues on the internal streams
+std::atomic<int> g_chunks{0};  // engram_set_overlap_chunks (0: the default)
+OverlapStreams g_overlap[64];
+
+// The internal streams and events of the current device (created on first use).
+OverlapStreams* overlap_streams() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  OverlapStreams& o = g_overlap[dev];
+  if (!o.ok) {
+    int lo_prio = 0, hi_prio = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo_prio, &hi_prio) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&o.hi, cudaStreamNonBlocking, hi_prio) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&o.lo, cudaStreamNonBlocking, lo_prio) != cudaSuccess ||
+        cudaEventCreateWithFlags(&o.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&o.proj, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&o.hi_done, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&o.lo_done, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    o.ok = true;
+  }
+  return &o;
+}
+
+// Chunks the pass runs in (1: one stream, the plain order).
+int overlap_chunks(int32_t B, int64_t M) {
+  if (g_debug.load() & ENGRAM_DEBUG_NO_OVERLAP) return 1;
+  if (g_events_on.load()) return 1;      // stage timing wants the stages one after another
+  static const int env = [] {
+    const char* v = getenv("ENGRAM_OVERLAP_CHUNKS");
+    return v != nullptr ? atoi(v) : -1;
+  }();
+  const int set = g_chunks.load();
+  int c = set > 0 ? set : (env >= 0 ? env : 1);
+  if (c > B) c = B;
+  if (c > 8) c = 8;
+  (void)M;
+  return c < 1 ? 1 : c;
+}
+
+// The CTA-pair projection serves this layer's dense prefill (bf16, 64-wide
+// rows, H % 256 == 0) unless a debug knob picks another engine.
+bool tc2_dense_supported(const engram_config* c) {
+  return (g_debug.load() & ENGRAM_DEBUG_TC_SINGLE_CTA) == 0 &&
+         tc_projection_supported(c->row_dim, c->hidden, c->dtype);
+}
+
+// a5-a9 of a prefill without state in `chunks` chunks of whole sequences on
+// the internal streams (see OverlapStreams); pp and cp describe the whole
+// batch.  The caller's stream s waits for everything before it goes on.
+engram_status forward_chunks(const engram_config* cfg, const ProjParams& pp0, const ConvParams& cp0, float* g,
+                             int chunks, OverlapStreams* o, cudaStream_t s) {
+  const int32_t B = cp0.B, T = cp0.T;
+  const size_t es = cfg->dtype == ENGRAM_F32 ? 4 : 2;
+  const int E = pp0.E, H = cfg->hidden, hc = cfg->hc_mult;
+  const int n_tiles = H / kTcTileN;
+  engram_status st = cuda_check(cudaEventRecord(o->fork, s), "fork");
+  if (st != ENGRAM_OK) return st;
+  st = cuda_check(cudaStreamWaitEvent(o->hi, o->fork, 0), "fork (projection stream)");
+  if (st != ENGRAM_OK) return st;
+  st = cuda_check(cudaStreamWaitEvent(o->lo, o->fork, 0), "fork (conv stream)");
+  if (st != ENGRAM_OK) return st;
+  for (int i = 0; i < chunks; ++i) {
+    const int32_t b0 = static_cast<int32_t>(static_cast<int64_t>(B) * i / chunks);
+    const int32_t b1 = static_cast<int32_t>(static_cast<int64_t>(B) * (i + 1) / chunks);
+    const int64_t m0 = static_cast<int64_t>(b0) * T, Mi = static_cast<int64_t>(b1 - b0) * T;
+    ProjParams pp = pp0;
+    pp.a_src = static_cast<const char*>(pp0.a_src) + m0 * E * es;
+    pp.a_rows = Mi * pp0.nh;
+    pp.hidden = static_cast<const char*>(pp0.hidden) + m0 * hc * H * es;
+    pp.V = static_cast<char*>(pp0.V) + m0 * H * es;
+    pp.partials = pp0.partials + m0 * hc * n_tiles;
+    pp.M = Mi;
+    pp.n_tiles = n_tiles;
+    pp.debug = g_debug.load();
+    st = cuda_check(launch_proj_tc2(pp, o->hi), "projection (tcgen05, CTA pairs)");
+    if (st != ENGRAM_OK) return st;
+    st = cuda_check(cudaEventRecord(o->proj, o->hi), "chunk event");
+    if (st != ENGRAM_OK) return st;
+    st = cuda_check(cudaStreamWaitEvent(o->lo, o->proj, 0), "chunk wait");
+    if (st != ENGRAM_OK) return st;
+    GateParams gp;
+    memset(&gp, 0, sizeof gp);
+    gp.partials = pp.partials;
+    gp.g = g + m0 * hc;
+    gp.M = Mi;
+    gp.hc = hc;
+    gp.n_tiles = n_tiles;
+    gp.H = H;
+    gp.rms_eps = cfg->rms_eps;
+    gp.gate_eps = cfg->gate_eps;
+    st = cuda_check(launch_gate(gp, o->lo), "gate");
+    if (st != ENGRAM_OK) return st;
+    ConvParams cp = cp0;
+    cp.V = pp.V;
+    cp.g = gp.g;
+    cp.Y = static_cast<char*>(cp0.Y) + m0 * hc * H * es;
+    cp.B = b1 - b0;
+    // beside the next chunk's projection: the slim form; the last chunk alone: the usual form
+    st = cuda_check(i + 1 < chunks ? launch_conv_slim(cp, o->lo) : launch_gated_conv(cp, o->lo), "gated conv");
+    if (st != ENGRAM_OK) return st;
+  }
+  st = cuda_check(cudaEventRecord(o->hi_done, o->hi), "join (projection stream)");
+  if (st != ENGRAM_OK) return st;
+  st = cuda_check(cudaEventRecord(o->lo_done, o->lo), "join (conv stream)");
+  if (st != ENGRAM_OK) return st;
+  st = cuda_check(cudaStreamWaitEvent(s, o->hi_done, 0), "join");
+  if (st != ENGRAM_OK) return st;
+  return cuda_check(cudaStreamWaitEvent(s, o->lo_done, 0), "join");
+}
+
 // Everything after the row gather (a5-a9 and the state advance), on a dense
 // e (rows == null; a_src = e [M, E]) or, for the fused-gather path, on the
 // table with the head-major absolute rows (a_src = table).  Shared by
@@ -339,6 +472,15 @@ engram_status forward_tail(const engram_config* cfg, const engram_weights* wts, 
     sa.T = T;
     sa.n_hist = n_hist;
   }
+  const int chunks = (state == nullptr && rows == nullptr && use_tc(cfg) && tc2_dense_supported(cfg) &&
+                      conv_slim_supported(cp))
+                         ? overlap_chunks(B, M)
+                         : 1;
+  if (chunks > 1) {
+    std::lock_guard<std::mutex> lock(g_overlap_mu);
+    OverlapStreams* o = overlap_streams();
+    if (o != nullptr) return forward_chunks(cfg, pp, cp, g, chunks, o, s);
+  }
   st = run_stage(cfg, pp, g, nullptr, s, state != nullptr ? &sa : nullptr);
   if (st != ENGRAM_OK) return st;
   record(g_events.before_conv, s);
@@ -411,6 +553,8 @@ size_t engram_last_error(char* buf, size_t n) {
 }
 
 void engram_set_debug(uint32_t flags) { g_debug.store(flags); }
+
+void engram_set_overlap_chunks(int32_t chunks) { g_chunks.store(chunks > 0 ? chunks : 0); }
 
 uint64_t engram_launch_count(void) { return g_launches.load(); }
 

@@ -207,6 +207,10 @@ struct ConvParams {
   FastDiv div_ring;         // ring_len, for the decode step (set by launch_gated_conv)
 };
 cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s);
+// The same conv in a form that fits beside the projection kernel on its SMs
+// (no shared memory, <= 88 registers at 128 threads): bf16, K = 4, no state.
+bool conv_slim_supported(const ConvParams& p);
+cudaError_t launch_conv_slim(const ConvParams& p, cudaStream_t s);
 // True when launch_gated_conv also writes the chunk's V/g rows into the state
 // rings (one decode step, T == 1), so no state advance follows.
 bool conv_writes_rings(const ConvParams& p);
@@ -362,29 +366,6 @@ __device__ __forceinline__ float gate_from_sums(float dot, float ssk, float ssq,
   const float rq = sqrtf(ssq * invH + rms_eps);
   const float s = dot / (rk * rq * sqrtf(static_cast<float>(H)));
   return gate_from_score(s, gate_eps);
-}
-
-// Gate of one (token, branch) from its n_tiles score partials
-// (sum K*nk*nq*Q, sum K^2, sum Q^2 per column tile), summed in tile order:
-//   s = dot / (sqrt(ssk/H + eps) sqrt(ssq/H + eps) sqrt(H)),  g = gate(s).
-__device__ __forceinline__ float gate_from_partials(const float4* part, int n_tiles, int H, float rms_eps,
-                                                    float gate_eps) {
-  float dot = 0.f, ssk = 0.f, ssq = 0.f;
-  int t = 0;
-  for (; t + 8 <= n_tiles; t += 8) {   // eight independent loads in flight
-    float4 v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = __ldg(part + t + u);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) { dot += v[u].x; ssk += v[u].y; ssq += v[u].z; }
-  }
-  for (; t < n_tiles; ++t) {
-    const float4 v = __ldg(part + t);
-    dot += v.x;
-    ssk += v.y;
-    ssq += v.z;
-  }
-  return gate_from_sums(dot, ssk, ssq, H, rms_eps, gate_eps);
 }
 
 }  // namespace engram

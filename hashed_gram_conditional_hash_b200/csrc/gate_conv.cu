@@ -21,12 +21,17 @@ namespace engram {
 namespace {
 
 // -------------------------------------------------------------- gate
-__global__ void gate_kernel(const __grid_constant__ GateParams p) {
+// G lanes per (token, branch): lane s of the group sums the score partials of
+// tiles s, s+G, s+2G, ... (so each load instruction of the warp covers whole
+// 128-byte lines of the partials), then the group adds its lanes' sums with
+// butterfly shuffles and its first lane forms the gate.
+template <int G>
+__global__ void __launch_bounds__(256) gate_kernel(const __grid_constant__ GateParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const StateIdsAdvance& st = p.state;
   if (st.pos != nullptr && i < st.B) {
-    // the streaming state's ids (M*hc >= B threads): the ring becomes the last
+    // the streaming state's ids (G*M*hc >= B threads): the ring becomes the last
     // n_hist ids of (old ring ++ chunk), ascending j reading index j + T >= j
     // before it is overwritten; pos advances by T
     const int b = static_cast<int>(i);
@@ -40,10 +45,38 @@ __global__ void gate_kernel(const __grid_constant__ GateParams p) {
     }
     st.pos[b] += st.T;
   }
-  if (i >= p.M * p.hc) return;
-  const float g = gate_from_partials(p.partials + i * p.n_tiles, p.n_tiles, p.H, p.rms_eps, p.gate_eps);
-  p.g[i] = g;
-  if (p.g_copy != nullptr) p.g_copy[i] = g;
+  const int64_t pair = i / G;                 // (token, branch) = m * hc + h
+  const int sub = static_cast<int>(i % G);
+  const bool live = pair < p.M * p.hc;
+  float dot = 0.f, ssk = 0.f, ssq = 0.f;
+  if (live) {
+    const float4* part = p.partials + pair * p.n_tiles;
+    int t = sub;
+    for (; t + 3 * G < p.n_tiles; t += 4 * G) {   // four independent loads in flight
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldg(part + t + u * G);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { dot += v[u].x; ssk += v[u].y; ssq += v[u].z; }
+    }
+    for (; t < p.n_tiles; t += G) {
+      const float4 v = __ldg(part + t);
+      dot += v.x;
+      ssk += v.y;
+      ssq += v.z;
+    }
+  }
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) {       // every lane takes part (dead ones add zeros)
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    ssk += __shfl_xor_sync(0xffffffffu, ssk, o);
+    ssq += __shfl_xor_sync(0xffffffffu, ssq, o);
+  }
+  if (live && sub == 0) {
+    const float g = gate_from_sums(dot, ssk, ssq, p.H, p.rms_eps, p.gate_eps);
+    p.g[pair] = g;
+    if (p.g_copy != nullptr) p.g_copy[pair] = g;
+  }
 }
 
 // -------------------------------------------------------------- gated conv
@@ -534,6 +567,89 @@ __global__ void __launch_bounds__((kTileC / CPL) * ENGRAM_MAX_HC) conv_tile_kern
   }
 }
 
+// The run form slimmed to run beside the projection kernel: no shared
+// memory and at most 88 registers at 128 threads, so one block fits in what
+// a projection CTA leaves free on its SM (bf16, K = 4, prefill without the
+// streaming state).  A thread owns 4 outputs of one residue class, 8
+// channels, one branch; it loads its 7 window rows and gates at once, keeps
+// its 32 taps packed as bf16, and forms each tap's U = g V when it is used,
+// in the same order of operations as the other forms (so the results are
+// the same bits).
+constexpr int kSlimThreads = 128;
+constexpr int kSlimRun = 4;
+
+__device__ __forceinline__ float2 tap_pair(const uint4& q, int i) {
+  // channels 2j and 2j+1 of the group's taps (uint4 j of the 8 x 4 layout), tap i
+  const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+  const uint32_t lo = words[i >> 1], hi = words[2 + (i >> 1)];
+  return (i & 1) ? make_float2(__uint_as_float(lo & 0xffff0000u), __uint_as_float(hi & 0xffff0000u))
+                 : make_float2(__uint_as_float(lo << 16), __uint_as_float(hi << 16));
+}
+
+__global__ void __launch_bounds__(kSlimThreads, 6) conv_slim_kernel(const __grid_constant__ ConvParams p) {
+  pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  constexpr int K = 4;
+  constexpr int RUN = kSlimRun;
+  constexpr int NW = RUN + K - 1;
+  const uint32_t gid = blockIdx.x * kSlimThreads + threadIdx.x;
+  if (gid >= p.div_b.d * static_cast<uint32_t>(p.B)) return;
+  const uint32_t b = fast_div(gid, p.div_b);
+  uint32_t rem = gid - b * p.div_b.d;
+  const uint32_t cls = fast_div(rem, p.div_cls);
+  rem -= cls * p.div_cls.d;
+  const uint32_t jr = fast_div(rem, p.div_run);
+  rem -= jr * p.div_run.d;
+  const int h = static_cast<int>(fast_div(rem, p.div_cg));
+  const int c = static_cast<int>(rem - h * p.div_cg.d) * 8;
+  const int t_first = static_cast<int>(cls + p.dil * (jr * RUN));
+  if (t_first >= p.T) return;
+  const int t0 = t_first - (K - 1) * p.dil;
+  const uint16_t* V = static_cast<const uint16_t*>(p.V);
+  const int64_t seq = static_cast<int64_t>(b) * p.T;
+  uint4 vraw[NW];
+  float gw[NW];
+#pragma unroll
+  for (int k = 0; k < NW; ++k) {
+    const int tp = t0 + k * p.dil;
+    if (tp >= 0 && tp < p.T) {
+      vraw[k] = __ldg(reinterpret_cast<const uint4*>(V + (seq + tp) * p.H + c));
+      gw[k] = __ldg(p.g + (seq + tp) * p.hc + h);
+    } else {
+      vraw[k] = make_uint4(0, 0, 0, 0);
+      gw[k] = 0.f;
+    }
+  }
+  uint4 wq[4];                                    // taps of the 8 channels, packed
+  const uint4* wsrc = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.conv_w) +
+                                                     (static_cast<int64_t>(h) * p.H + c) * K);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) wq[j] = __ldg(wsrc + j);
+  uint16_t* yp = static_cast<uint16_t*>(p.Y) + ((seq + t_first) * p.hc + h) * p.H + c;
+  const int64_t ys = static_cast<int64_t>(p.dil) * p.hc * p.H;
+#pragma unroll
+  for (int q = 0; q < RUN; ++q) {
+    if (t_first + q * p.dil >= p.T) break;
+    float2 acc[4];
+    float2 u[K][4];
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      float2 v[4];
+      Pair8<uint16_t>::unpack(vraw[q + i], v);
+      const float2 g2 = make_float2(gw[q + i], gw[q + i]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) u[i][j] = __fmul2_rn(g2, v[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 a = u[K - 1][j];
+#pragma unroll
+      for (int i = 0; i < K; ++i) a = __ffma2_rn(tap_pair(wq[j], i), u[i][j], a);
+      acc[j] = a;
+    }
+    Pair8<uint16_t>::store(yp + q * ys, acc);
+  }
+}
+
 // One decode step (T = 1) with the streaming state, K = 4 taps, bfloat16:
 // block (group of kStepSeq sequences, 256-channel slice), one warp per
 // branch, 8 channels per lane.  A lane loads its taps once for the group,
@@ -729,8 +845,20 @@ int grid_cap() { return num_sms() * 8; }
 cudaError_t launch_gate(const GateParams& p, cudaStream_t s) {
   const int64_t n = p.M * p.hc;
   if (n <= 0) return cudaSuccess;
-  // small blocks: the few gates of a step spread over every SM
-  launch_k(gate_kernel, dim3(static_cast<unsigned>((n + 63) / 64)), dim3(64), 0, s, p);
+  // lanes per (token, branch): the partials' tile count rounded up to a
+  // power of two, at most 8
+  const int G = p.n_tiles >= 8 ? 8 : p.n_tiles >= 4 ? 4 : p.n_tiles >= 2 ? 2 : 1;
+  int64_t threads = n * G;
+  if (p.state.pos != nullptr && threads < p.state.B) threads = p.state.B;
+  const int64_t blocks = (threads + 255) / 256;
+  if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(blocks));
+  switch (G) {
+    case 8: launch_k(gate_kernel<8>, grid, dim3(256), 0, s, p); break;
+    case 4: launch_k(gate_kernel<4>, grid, dim3(256), 0, s, p); break;
+    case 2: launch_k(gate_kernel<2>, grid, dim3(256), 0, s, p); break;
+    default: launch_k(gate_kernel<1>, grid, dim3(256), 0, s, p); break;
+  }
   return cudaGetLastError();
 }
 
@@ -745,6 +873,27 @@ bool tile_form(const ConvParams& p) {
 bool conv_writes_rings(const ConvParams& p) {
   return p.T == 1 && p.pos != nullptr && p.v_ring != nullptr && p.g_ring != nullptr && p.K == 4 &&
          p.conv_w != nullptr && p.dtype == ENGRAM_BF16 && p.H % kTileC == 0 && p.hc <= ENGRAM_MAX_HC;
+}
+
+bool conv_slim_supported(const ConvParams& p) {
+  return p.K == 4 && p.conv_w != nullptr && p.dtype == ENGRAM_BF16 && p.v_ring == nullptr && p.H % 8 == 0 &&
+         p.B > 0 && p.T > 0;
+}
+
+cudaError_t launch_conv_slim(const ConvParams& p, cudaStream_t s) {
+  if (!conv_slim_supported(p)) return cudaErrorInvalidValue;
+  const int64_t rpc = (p.T + static_cast<int64_t>(p.dil) * kSlimRun - 1) / (static_cast<int64_t>(p.dil) * kSlimRun);
+  const int64_t nthreads = static_cast<int64_t>(p.B) * p.dil * rpc * p.hc * (p.H / 8);
+  const int64_t blocks = (nthreads + kSlimThreads - 1) / kSlimThreads;
+  if (blocks * kSlimThreads > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit thread ids
+  ConvParams q = p;
+  const uint32_t per_run = static_cast<uint32_t>(p.hc * (p.H / 8));
+  q.div_cg = make_fastdiv(static_cast<uint32_t>(p.H / 8));
+  q.div_run = make_fastdiv(per_run);
+  q.div_cls = make_fastdiv(static_cast<uint32_t>(rpc) * per_run);
+  q.div_b = make_fastdiv(static_cast<uint32_t>(p.dil) * static_cast<uint32_t>(rpc) * per_run);
+  launch_k(conv_slim_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kSlimThreads), 0, s, q);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gated_conv(const ConvParams& p, cudaStream_t s) {

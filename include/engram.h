@@ -156,7 +156,26 @@ uint64_t engram_launch_count(void);
  * with programmatic dependent launch (which lets a kernel be scheduled while
  * its predecessor on the stream finishes). */
 #define ENGRAM_DEBUG_NO_PDL 0x10u
+/* ENGRAM_DEBUG_NO_OVERLAP runs a prefill's stages one after another on the
+ * caller's stream instead of in sequence chunks whose gate and conv overlap
+ * the next chunk's projection on two internal streams. */
+#define ENGRAM_DEBUG_NO_OVERLAP 0x20u
 void engram_set_debug(uint32_t flags);
+
+/* Sequence chunks of a prefill (process-wide; explainer §4.4 overlaps the
+ * memory-side work of the layer with the dense compute).  With chunks > 1,
+ * engram_forward and engram_forward_gathered, when the prefill (no state)
+ * runs on the CTA-pair projection with the bf16 K = 4 conv, split the batch
+ * into up to `chunks` groups of whole sequences: each group's projection on
+ * a high-priority internal stream, its gate and conv on a low-priority one,
+ * so one group's gate and conv run beside the next group's projection.  The
+ * results are the same bits as with chunks = 1.  The first such call on a
+ * device creates the two internal streams and four events it uses (make it
+ * before any stream capture); the caller's stream waits for both streams
+ * before its next work, and calls from several host threads enqueue one at
+ * a time.  chunks <= 0 restores the default (1, or the ENGRAM_OVERLAP_CHUNKS
+ * environment variable); values above 8 or above B are clipped. */
+void engram_set_overlap_chunks(int32_t chunks);
 
 /* Which projection engine engram_forward / engram_gate_fuse use for cfg under
  * the current debug flags: ENGRAM_ENGINE_TCGEN05 (tensor cores, bfloat16,

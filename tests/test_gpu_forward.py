@@ -23,8 +23,9 @@ ENGINE_FLAGS = {"auto": 0, "simt": L.DEBUG_FORCE_SIMT, "fused": L.DEBUG_FUSED_GA
                 "single_cta": L.DEBUG_TC_SINGLE_CTA}
 
 
-def _run(p, engine="auto", conv_w=None):
+def _run(p, engine="auto", conv_w=None, chunks=1):
     L.engram_set_debug(ENGINE_FLAGS[engine])
+    L.engram_set_overlap_chunks(chunks)
     try:
         layer = EngramLayer.from_params(p)
         if conv_w is not None:
@@ -35,6 +36,7 @@ def _run(p, engine="auto", conv_w=None):
         return y
     finally:
         L.engram_set_debug(0)
+        L.engram_set_overlap_chunks(0)
 
 
 SMALL = [
@@ -88,10 +90,10 @@ def test_forward_full_size_sampled(name):
     Yref, _, _, _ = oracle_at(p, pos)
     bi = torch.tensor([b for b, _ in pos], device=DEV)
     ti = torch.tensor([t for _, t in pos], device=DEV)
-    for engine in ("auto", "single_cta"):
-        y = _run(p, engine)
+    for engine, chunks in (("auto", 1), ("single_cta", 1), ("auto", 4)):
+        y = _run(p, engine, chunks=chunks)
         err = rel_err(y[bi, ti].double().cpu().numpy(), Yref)
-        assert err <= TOL[w.dtype], (engine, err)
+        assert err <= TOL[w.dtype], (engine, chunks, err)
         del y
 
 
@@ -134,6 +136,34 @@ def test_forward_branch_with_zero_hidden_gates_one_half():
     for engine in ("auto", "simt"):
         y = _run(p, engine)
         assert rel_err(y.double().cpu().numpy(), ref["Y"]) <= TOL["bf16"], engine
+
+
+OVERLAP = [
+    (dict(B=2, T=300, hidden=512, hc_mult=4), 2),
+    (dict(B=5, T=130, hidden=256, hc_mult=2, orders=(2, 3, 4), dilation=4), 3),  # uneven chunks
+    (dict(B=3, T=77), 8),                                                         # clipped to B
+    (dict(B=4, T=40, hidden=768, hc_mult=3, dilation=9), 2),                     # long halo, short chunks
+]
+
+
+@pytest.mark.parametrize("kw,chunks", OVERLAP, ids=[str(i) for i in range(len(OVERLAP))])
+def test_forward_overlapped_chunks_equal_plain(kw, chunks):
+    # the pass in sequence chunks whose gate and conv overlap the next chunk's
+    # projection on two streams: the same kernels per element, so the same bits
+    w = W.small_workload(**kw)
+    p = device_params(w)
+    plain = _run(p, chunks=1)
+    y = _run(p, chunks=chunks)
+    assert torch.equal(y, plain)
+    assert rel_err(y.double().cpu().numpy(), oracle_forward_full(p)["Y"]) <= TOL[w.dtype]
+
+
+def test_forward_overlapped_chunks_model_shaped():
+    w = W.CONFIGS["model_bf16"]
+    p = device_params(w)
+    plain = _run(p, chunks=1)
+    for chunks in (2, 4):
+        assert torch.equal(_run(p, chunks=chunks), plain), chunks
 
 
 def test_forward_split_value_tail_tiles():
