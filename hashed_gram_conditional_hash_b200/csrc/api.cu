@@ -198,7 +198,7 @@ engram_status run_projection(const engram_config* c, ProjParams* pp, cudaStream_
 
 // Projection followed by the stand-alone gate kernel (engram_gate_fuse).
 engram_status run_stage(const engram_config* c, ProjParams pp, float* g, float* g_copy,
-                        cudaStream_t s, const StateIdsAdvance* state_ids = nullptr) {
+                        cudaStream_t s, const StateIdsAdvance* state_ids = nullptr, bool trigger_early = false) {
   engram_status st = run_projection(c, &pp, s);
   if (st != ENGRAM_OK) return st;
   GateParams gp;
@@ -213,6 +213,7 @@ engram_status run_stage(const engram_config* c, ProjParams pp, float* g, float* 
   gp.H = c->hidden;
   gp.rms_eps = c->rms_eps;
   gp.gate_eps = c->gate_eps;
+  gp.trigger_early = trigger_early ? 1 : 0;
   return cuda_check(launch_gate(gp, s), "gate");
 }
 
@@ -445,7 +446,7 @@ engram_status forward_tail(const engram_config* cfg, const engram_weights* wts, 
     cp.v_ring = state->v_ring;
     cp.g_ring = state->g_ring;
     cp.pos = state->pos;
-    cp.pos_lag = T;  // advanced by the gate kernel
+    cp.pos_lag = T;  // advanced by the hash kernel
     cp.ring_len = state->ring_len;
   }
   cp.B = B;
@@ -460,8 +461,8 @@ engram_status forward_tail(const engram_config* cfg, const engram_weights* wts, 
   StateIdsAdvance sa;
   memset(&sa, 0, sizeof sa);
   if (state != nullptr) {
+    sa.active = 1;
     sa.id_ring = state->id_ring;
-    sa.pos = state->pos;
     sa.ids = ids;
     sa.lookup = wts->lookup;
     sa.status = dev_status;
@@ -481,7 +482,11 @@ engram_status forward_tail(const engram_config* cfg, const engram_weights* wts, 
     OverlapStreams* o = overlap_streams();
     if (o != nullptr) return forward_chunks(cfg, pp, cp, g, chunks, o, s);
   }
-  st = run_stage(cfg, pp, g, nullptr, s, state != nullptr ? &sa : nullptr);
+  // before the decode conv step the gate lets that step start early (it loads
+  // the state's pos and ring rows, which no kernel of this call after the
+  // hash writes, while the gates are formed)
+  st = run_stage(cfg, pp, g, nullptr, s, state != nullptr ? &sa : nullptr,
+                 state != nullptr && conv_writes_rings(cp));
   if (st != ENGRAM_OK) return st;
   record(g_events.before_conv, s);
   st = cuda_check(launch_gated_conv(cp, s), "gated conv");
@@ -834,6 +839,7 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   hp.lookup = wts->lookup;
   hp.raw_vocab = wts->raw_vocab;
   hp.history = state != nullptr ? state->id_ring : nullptr;
+  hp.pos_advance = state != nullptr ? state->pos : nullptr;   // pos += T, first kernel of the call
   hp.rows_out = fused ? rows : nullptr;
   hp.idx_out = nullptr;
   hp.ld_rows = ld;

@@ -42,6 +42,7 @@ struct HashParams {
   const int64_t* history;   // [B, n_hist] or null (then pad_id)
   int64_t* idx_out;         // [B*T, nh] int64 or null
   int32_t* rows_out;        // [nh, ld_rows] absolute table rows (int32) or null
+  int64_t* pos_advance;     // [B] streaming state's pos: += T by the kernel, or null
   uint32_t* status;
   int64_t raw_vocab;
   int64_t vocab;
@@ -162,11 +163,11 @@ cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s);
 
 // Gate finalisation (a6 reduction + a7): g[m, h] from the partials.
 // The streaming state's id bookkeeping of one chunk, done by the gate kernel
-// (after the hash has read the ring, before the conv reads pos): the id ring
-// takes the chunk's last ids and pos advances by T.
+// (after the hash has read the ring): the id ring takes the chunk's last ids.
+// (pos advances in the hash kernel, the first of the call.)
 struct StateIdsAdvance {
+  int32_t active;           // 0: no streaming state
   int64_t* id_ring;         // [B, n_hist]
-  int64_t* pos;             // [B]; null: nothing to do
   const int64_t* ids;       // [B, T] chunk ids (raw when lookup != null)
   const int64_t* lookup;    // [raw_vocab] or null
   uint32_t* status;
@@ -181,7 +182,8 @@ struct GateParams {
   int64_t M;
   int32_t hc, n_tiles, H;
   float rms_eps, gate_eps;
-  StateIdsAdvance state;    // state.pos == null: no streaming state
+  StateIdsAdvance state;    // state.active == 0: no streaming state
+  int32_t trigger_early;    // let the next kernel (the decode conv step) start at once
 };
 cudaError_t launch_gate(const GateParams& p, cudaStream_t s);
 

@@ -28,12 +28,15 @@ namespace {
 template <int G>
 __global__ void __launch_bounds__(256) gate_kernel(const __grid_constant__ GateParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  // the decode conv step reads only earlier calls' state before its own wait,
+  // so it may be scheduled now and load that state while the gates are formed
+  if (p.trigger_early) pdl_trigger();
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const StateIdsAdvance& st = p.state;
-  if (st.pos != nullptr && i < st.B) {
+  if (st.active && i < st.B) {
     // the streaming state's ids (G*M*hc >= B threads): the ring becomes the last
     // n_hist ids of (old ring ++ chunk), ascending j reading index j + T >= j
-    // before it is overwritten; pos advances by T
+    // before it is overwritten
     const int b = static_cast<int>(i);
     int64_t* ring = st.id_ring + static_cast<int64_t>(b) * st.n_hist;
     const int64_t base = static_cast<int64_t>(b) * st.T;
@@ -43,7 +46,6 @@ __global__ void __launch_bounds__(256) gate_kernel(const __grid_constant__ GateP
                                 : checked_id(__ldg(st.ids + base + (src - st.n_hist)), st.lookup, st.raw_vocab,
                                              st.vocab, st.pad_id, st.status);
     }
-    st.pos[b] += st.T;
   }
   const int64_t pair = i / G;                 // (token, branch) = m * hc + h
   const int sub = static_cast<int>(i % G);
@@ -652,19 +654,19 @@ __global__ void __launch_bounds__(kSlimThreads, 6) conv_slim_kernel(const __grid
 
 // One decode step (T = 1) with the streaming state, K = 4 taps, bfloat16:
 // block (group of kStepSeq sequences, 256-channel slice), one warp per
-// branch, 8 channels per lane.  A lane loads its taps once for the group,
-// then, for every sequence of the group at once, its 16-byte piece of V(t),
-// the step's gate and pos; turns pos into the ring rows of the taps at
-// t - 3 dil, t - 2 dil, t - dil (the ring holds (K-1) dil + 1 >= 3 dil + 1
-// positions, slot = position mod ring length, by invariant-divisor
-// multiplication) and loads its pieces of those rows and their gates, so that
-// each lane has every sequence's loads in flight together; then it stores 8
-// channels of Y per sequence.  No block barrier.  The same kernel is the
-// step's state advance: the branch-0 warp writes V(t) and lanes 0 write g(t)
-// into t's slot, which no tap of this step reads.
+// branch, 8 channels per lane.  Before its programmatic-launch wait (the
+// gate kernel lets this grid start early) a lane loads its taps once for the
+// group, every sequence's pos (advanced by this call's hash kernel), turns
+// pos into the ring rows of the taps at t - 3 dil, t - 2 dil, t - dil (the
+// ring holds (K-1) dil + 1 >= 3 dil + 1 positions, slot = position mod ring
+// length, by invariant-divisor multiplication) and loads its pieces of those
+// rows and their gates, all written by earlier calls; after the wait, its
+// 16-byte piece of V(t) and the step's gate; then it stores 8 channels of Y
+// per sequence.  No block barrier.  The same kernel is the step's state
+// advance: the branch-0 warp writes V(t) and lanes 0 write g(t) into t's
+// slot, which no tap of this step reads.
 template <int S>
 __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __grid_constant__ ConvParams p) {
-  pdl_wait();  // the previous kernel on the stream has finished (PDL)
   constexpr int K = 4;
   const int tid = static_cast<int>(threadIdx.x);
   const int h = tid >> 5, lane = tid & 31;
@@ -676,21 +678,16 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __g
   float* gr = const_cast<float*>(p.g_ring);
   uint4 raw[S][K];
   float gg[S][K];
+  // Before the wait: what no kernel of this call after the hash writes.  pos
+  // was advanced by this call's hash kernel (finished before the projection
+  // began), the ring rows of the taps by earlier calls, the taps are
+  // weights; the gate kernel lets this grid start while it runs, so these
+  // dependent loads (pos, then the rows it selects) overlap the gates.
+  // Read through L2 (the state is written by other grids).
   int64_t P[S];
-  // what does not depend on the ring, for the whole group
+  int64_t row_t[S];
 #pragma unroll
-  for (int s = 0; s < S; ++s) {
-    const int b = b0 + s;
-    if (b < p.B) {
-      raw[s][K - 1] = __ldg(reinterpret_cast<const uint4*>(V + static_cast<int64_t>(b) * p.H + c));
-      gg[s][K - 1] = __ldg(p.g + static_cast<int64_t>(b) * p.hc + h);
-      P[s] = __ldg(p.pos + b) - p.pos_lag;          // position of this step's token
-    } else {
-      raw[s][K - 1] = make_uint4(0, 0, 0, 0);
-      gg[s][K - 1] = 0.f;
-      P[s] = -1;
-    }
-  }
+  for (int s = 0; s < S; ++s) P[s] = (b0 + s < p.B) ? __ldcg(p.pos + b0 + s) - p.pos_lag : -1;
   float2 w2[4][K];                                // [channel pair][tap]
   {
     float w[8][K];
@@ -700,11 +697,9 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __g
 #pragma unroll
       for (int i = 0; i < K; ++i) w2[j][i] = make_float2(w[2 * j][i], w[2 * j + 1][i]);
   }
-  // the ring rows of the taps, for the whole group
-  int64_t row_t[S];
 #pragma unroll
   for (int s = 0; s < S; ++s) {
-    const int64_t Ps = P[s];
+    const int64_t Ps = P[s];                        // position of this step's token (-1: no sequence)
     const int64_t slot_t = (Ps >= 0 && Ps < INT32_MAX)
                                ? static_cast<int64_t>(Ps - static_cast<int64_t>(fast_div(static_cast<uint32_t>(Ps), p.div_ring)) *
                                                               p.ring_len)
@@ -718,12 +713,24 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __g
       if (slot < 0) slot += p.ring_len;
       if (Ps - back >= 0) {                         // also false past the last sequence (P = -1)
         const int64_t row = ring0 + slot;
-        raw[s][i] = __ldg(reinterpret_cast<const uint4*>(vr + row * p.H + c));
-        gg[s][i] = __ldg(gr + row * p.hc + h);
+        raw[s][i] = __ldcg(reinterpret_cast<const uint4*>(vr + row * p.H + c));
+        gg[s][i] = __ldcg(gr + row * p.hc + h);
       } else {
         raw[s][i] = make_uint4(0, 0, 0, 0);
         gg[s][i] = 0.f;
       }
+    }
+  }
+  pdl_wait();  // the gate kernel (and so the projection) has finished: V(t), g(t)
+#pragma unroll
+  for (int s = 0; s < S; ++s) {
+    const int b = b0 + s;
+    if (b < p.B) {
+      raw[s][K - 1] = __ldg(reinterpret_cast<const uint4*>(V + static_cast<int64_t>(b) * p.H + c));
+      gg[s][K - 1] = __ldg(p.g + static_cast<int64_t>(b) * p.hc + h);
+    } else {
+      raw[s][K - 1] = make_uint4(0, 0, 0, 0);
+      gg[s][K - 1] = 0.f;
     }
   }
 #pragma unroll
@@ -849,7 +856,7 @@ cudaError_t launch_gate(const GateParams& p, cudaStream_t s) {
   // power of two, at most 8
   const int G = p.n_tiles >= 8 ? 8 : p.n_tiles >= 4 ? 4 : p.n_tiles >= 2 ? 2 : 1;
   int64_t threads = n * G;
-  if (p.state.pos != nullptr && threads < p.state.B) threads = p.state.B;
+  if (p.state.active && threads < p.state.B) threads = p.state.B;
   const int64_t blocks = (threads + 255) / 256;
   if (blocks > INT32_MAX) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(blocks));

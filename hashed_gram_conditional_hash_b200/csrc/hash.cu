@@ -27,6 +27,8 @@ __device__ __forceinline__ int64_t load_id(const HashParams& p, int64_t raw) {
 
 __global__ void __launch_bounds__(256) hash_kernel(const __grid_constant__ HashParams p) {
   pdl_wait();  // the previous kernel on the stream has finished (PDL)
+  // the streaming state's pos counts this chunk (the call's first kernel does it)
+  if (p.pos_advance != nullptr && blockIdx.x == 0 && threadIdx.x == 0) p.pos_advance[blockIdx.y] += p.T;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int b = blockIdx.y;
@@ -145,6 +147,8 @@ __device__ __forceinline__ void hash_gather_body(const HashGatherParams& g) {
   if (g.wprod != nullptr)   // the RMSNorm weight products of the score, for the projection
     for (int i = gtid; i < g.n_w; i += static_cast<int>(gridDim.x * blockDim.x))
       g.wprod[i] = bf16_to_f32(__ldg(g.nk + i)) * bf16_to_f32(__ldg(g.nq + i));
+  // the streaming state's pos counts this chunk (the grid has at least B threads)
+  if (p.pos_advance != nullptr && gtid < p.B && blockIdx.y == 0) p.pos_advance[gtid] += p.T;
   // rows of e (B*T*nh) stay below 2^31 (checked by the launcher): 32-bit math
   const int total = p.B * p.T * p.nh;
   const int q0 = (gtid >> 5) * ROWS;
@@ -250,6 +254,8 @@ __device__ __forceinline__ void hash_gather_w32_body(const HashGatherParams& g, 
   if (g.wprod != nullptr)   // the RMSNorm weight products of the score, for the projection
     for (int i = gtid; i < g.n_w; i += static_cast<int>(gridDim.x * blockDim.x))
       g.wprod[i] = bf16_to_f32(__ldg(g.nk + i)) * bf16_to_f32(__ldg(g.nq + i));
+  // the streaming state's pos counts this chunk (the grid has at least B threads)
+  if (p.pos_advance != nullptr && gtid < p.B && blockIdx.y == 0) p.pos_advance[gtid] += p.T;
   const int M = p.B * p.T;
   const int total = M * p.nh;                       // < 2^31 (checked by the launcher)
   const int qw = (gtid >> 5) * (32 * NC);           // first row of the warp
