@@ -289,6 +289,7 @@ def run_ours(args, rank, world, device):
         w = w.replace(decode_calls=args.decode_calls)
     peaks, peak_kind = load_peaks()
     L.engram_set_overlap_chunks(args.overlap_chunks)
+    L.engram_set_debug(args.debug_flags)
     p = W.make_params(w, device)
     layer = EngramLayer.from_params(p)
     engine = "tcgen05" if L.engram_projection_engine(layer.cfg) == L.ENGINE_TCGEN05 else "simt"
@@ -766,6 +767,8 @@ def main():
     ap.add_argument("--ref-step-s", type=float, default=3.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--debug-flags", type=lambda x: int(x, 0), default=0,
+                    help="library comparison knobs (ENGRAM_DEBUG_* of engram.h), e.g. 0x40")
     ap.add_argument("--overlap-chunks", type=int, default=0,
                     help="prefill in this many sequence chunks whose gate and conv overlap the next "
                          "chunk's projection (0: the library default)")

@@ -24,6 +24,7 @@ ENGRAM_F32, ENGRAM_BF16 = 0, 1
 STATUS_ID_RANGE, STATUS_ROW_RANGE, STATUS_TIMEOUT = 0x1, 0x2, 0x4
 DEBUG_FORCE_TIMEOUT, DEBUG_FORCE_SIMT, DEBUG_FUSED_GATHER, DEBUG_TC_SINGLE_CTA, DEBUG_NO_PDL = 0x1, 0x2, 0x4, 0x8, 0x10
 DEBUG_NO_OVERLAP = 0x20
+DEBUG_TILE_MBLOCK_ORDER = 0x40
 STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_CUDA",
                 4: "ERR_TIMEOUT", 5: "ERR_ID_RANGE"}
 

@@ -46,10 +46,16 @@
 // Every wait is bounded; an abort raises the flag in both CTAs; no multicast
 // loads are used anywhere (only the commit arrives on both CTAs' barriers).
 //
-// Tiles run M-block-major (an M-block's key tiles, then its value tiles) over
-// a persistent grid of as many pairs as fit; when the last round of pairs
-// would be at most half full, that many value tiles from the end run as twice
-// as many 256 x 128 tiles (N = 128 MMA, 64 weight rows per CTA).  The key
+// Tiles run over a persistent grid of as many pairs as fit, in groups of
+// M-blocks whose rows of e fill about 32 MB, N-tile by N-tile within a group:
+// a weight tile then serves the group's M-blocks while it is in L2, and the
+// group's rows of e stay in L2 for all its N-tiles (M-block-major order, all
+// N-tiles of one M-block before the next, re-read the weights from HBM once
+// they outgrew L2: 8.8 GB of DRAM reads per HBM-scale launch against 2.5 GB
+// of operands and hidden state).  When the last round of pairs would be at
+// most half full, that many value tiles from the end (the last group's last
+// N-tiles) run as twice as many 256 x 128 tiles (N = 128 MMA, 64 weight rows
+// per CTA).  The key
 // epilogue takes norm_key * norm_query from a per-call fp32 table when given.
 #include <cuda.h>
 
@@ -91,6 +97,10 @@ struct Tc2Params {
   // of M-block mb0 on) run at the end as 2 * n_split half-width tiles, so that
   // the last round of pairs is not left mostly idle
   int32_t nk_tiles, n_split, mb0, vb0;
+  // with no split tail: tiles run in groups of `group_mb` M-blocks, N-tile by
+  // N-tile within a group (each weight tile serves the group's M-blocks while
+  // it is in L2; the group's rows of e stay in L2 for all its N-tiles)
+  int32_t group_mb, m_blocks;
   int64_t num_tiles;                         // pair tiles
   uint64_t timeout_ns;
   int32_t force_timeout;
@@ -112,6 +122,31 @@ __device__ __forceinline__ Tile tile_at(const Tc2Params& tp, int64_t t) {
   const int64_t n_full = tp.num_tiles - 2 * static_cast<int64_t>(tp.n_split);
   x.half = false;
   x.width = kBN;
+  if (tp.group_mb > 0) {                   // grouped order
+    const int64_t n_full = tp.num_tiles - 2 * static_cast<int64_t>(tp.n_split);
+    int64_t f = t;                         // index of the full tile in grouped order
+    int hf = -1;                           // half of a split tile (the last n_split full tiles)
+    if (t >= n_full) {
+      f = n_full + ((t - n_full) >> 1);
+      hf = static_cast<int>((t - n_full) & 1);
+    }
+    const int64_t per_group = static_cast<int64_t>(tp.group_mb) * nn;
+    const int64_t grp = f / per_group;
+    const int64_t in = f - grp * per_group;
+    const int64_t mb_first = grp * tp.group_mb;
+    const int64_t gm = min(static_cast<int64_t>(tp.group_mb), tp.m_blocks - mb_first);   // M-blocks in the group
+    const int n = static_cast<int>(in / gm);
+    x.mb = mb_first + (in - static_cast<int64_t>(n) * gm);
+    x.is_v = n >= nk;
+    x.kt = x.is_v ? 0 : n;
+    x.col0 = (x.is_v ? n - nk : n) * kBN;
+    if (hf >= 0) {                         // (value tiles: checked on the host)
+      x.half = true;
+      x.width = kBN / 2;
+      x.col0 += hf * (kBN / 2);
+    }
+    return x;
+  }
   int r;                                   // index inside the M-block (keys, then values)
   if (t >= n_full) {                       // half-width value tiles
     const int64_t i = t - n_full;
@@ -606,6 +641,21 @@ cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s) {
   tp.mb0 = static_cast<int32_t>(first_split / tp.nv_tiles);
   tp.vb0 = static_cast<int32_t>(first_split % tp.nv_tiles);
   tp.num_tiles = full + tp.n_split;                                // n_split full tiles become 2 * n_split
+  // grouped order when no tail is split: M-blocks whose rows of e fill about
+  // 32 MB per group (half of one die's L2 partition)
+  tp.m_blocks = static_cast<int32_t>(m2);
+  tp.group_mb = 0;
+  if (!(p.debug & ENGRAM_DEBUG_TILE_MBLOCK_ORDER)) {
+    const int64_t rows_bytes = static_cast<int64_t>(2 * kBM) * p.E * 2;          // one M-block of e
+    int64_t g = (static_cast<int64_t>(32) << 20) / (rows_bytes > 0 ? rows_bytes : 1);
+    if (g < 1) g = 1;
+    if (g > m2) g = m2;
+    const int64_t groups = (m2 + g - 1) / g;
+    g = (m2 + groups - 1) / groups;          // groups of (nearly) equal size
+    // the split tail must be value tiles: the last group's last N-tiles
+    const int64_t g_last = m2 - ((m2 - 1) / g) * g;
+    if (tp.n_split <= tp.nv_tiles * g_last) tp.group_mb = static_cast<int32_t>(g);
+  }
   tp.force_timeout = (p.debug & ENGRAM_DEBUG_FORCE_TIMEOUT) ? 1 : 0;
   tp.timeout_ns = tp.force_timeout ? 20000000ull : 2000000000ull;
   // two K-blocks per TMA box when the head count allows it

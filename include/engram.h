@@ -160,6 +160,10 @@ uint64_t engram_launch_count(void);
  * caller's stream instead of in sequence chunks whose gate and conv overlap
  * the next chunk's projection on two internal streams. */
 #define ENGRAM_DEBUG_NO_OVERLAP 0x20u
+/* ENGRAM_DEBUG_TILE_MBLOCK_ORDER runs the CTA-pair projection's tiles M-block
+ * by M-block (every N-tile of one 256-row block before the next) instead of in
+ * groups of M-blocks, N-tile by N-tile within a group. */
+#define ENGRAM_DEBUG_TILE_MBLOCK_ORDER 0x40u
 void engram_set_debug(uint32_t flags);
 
 /* Sequence chunks of a prefill (process-wide; explainer §4.4 overlaps the

@@ -20,7 +20,7 @@ DEV = "cuda"
 
 ENGINE_FLAGS = {"auto": 0, "simt": L.DEBUG_FORCE_SIMT, "fused": L.DEBUG_FUSED_GATHER,
                 "simt_fused": L.DEBUG_FORCE_SIMT | L.DEBUG_FUSED_GATHER,
-                "single_cta": L.DEBUG_TC_SINGLE_CTA}
+                "single_cta": L.DEBUG_TC_SINGLE_CTA, "mblock_order": L.DEBUG_TILE_MBLOCK_ORDER}
 
 
 def _run(p, engine="auto", conv_w=None, chunks=1):
@@ -177,6 +177,17 @@ def test_forward_split_value_tail_tiles():
     # the same rows through the single-CTA engine (no tile split)
     d = _run(p, "single_cta").double()
     assert (y.double() - d).abs().max().item() <= 1e-2 * d.abs().max().item()
+
+
+@pytest.mark.parametrize("kw", [dict(B=2, T=256, hidden=2048, hc_mult=4),   # split value tail
+                                dict(B=4, T=300, hidden=512, hc_mult=4),    # several groups of M-blocks
+                                dict(B=3, T=77)])
+def test_forward_tile_orders_agree(kw):
+    # the projection's tiles in groups of M-blocks (default) or M-block by
+    # M-block: every output element is the same computation, so the same bits
+    w = W.small_workload(**kw)
+    p = device_params(w)
+    assert torch.equal(_run(p), _run(p, "mblock_order"))
 
 
 def test_forward_engines_agree():
