@@ -47,7 +47,7 @@
 // loads are used anywhere (only the commit arrives on both CTAs' barriers).
 //
 // Tiles run over a persistent grid of as many pairs as fit, in groups of
-// M-blocks whose rows of e fill about 32 MB, N-tile by N-tile within a group:
+// M-blocks whose rows of e fill about 16 MB, N-tile by N-tile within a group:
 // a weight tile then serves the group's M-blocks while it is in L2, and the
 // group's rows of e stay in L2 for all its N-tiles (M-block-major order, all
 // N-tiles of one M-block before the next, re-read the weights from HBM once
@@ -69,6 +69,10 @@ namespace {
 using namespace tc;
 
 constexpr int kBM = 128;                    // token rows per CTA (pair: 256)
+// rows of e per group of M-blocks in the tile order (measured on the
+// HBM-scale workload, ms per step: 16 MB 4.66, 32 MB 4.72, 64 MB 5.11;
+// M-block by M-block 5.38 on another box against 5.02 for 32 MB)
+constexpr int64_t kTileGroupBytes = static_cast<int64_t>(16) << 20;
 constexpr int kBN = 256;                    // output columns per pair tile
 constexpr int kBNh = kBN / 2;               // weight rows per CTA
 constexpr int kBK = 64;
@@ -641,13 +645,13 @@ cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s) {
   tp.mb0 = static_cast<int32_t>(first_split / tp.nv_tiles);
   tp.vb0 = static_cast<int32_t>(first_split % tp.nv_tiles);
   tp.num_tiles = full + tp.n_split;                                // n_split full tiles become 2 * n_split
-  // grouped order when no tail is split: M-blocks whose rows of e fill about
-  // 32 MB per group (half of one die's L2 partition)
+  // grouped order: M-blocks whose rows of e fill about kTileGroupBytes per
+  // group
   tp.m_blocks = static_cast<int32_t>(m2);
   tp.group_mb = 0;
   if (!(p.debug & ENGRAM_DEBUG_TILE_MBLOCK_ORDER)) {
     const int64_t rows_bytes = static_cast<int64_t>(2 * kBM) * p.E * 2;          // one M-block of e
-    int64_t g = (static_cast<int64_t>(32) << 20) / (rows_bytes > 0 ? rows_bytes : 1);
+    int64_t g = kTileGroupBytes / (rows_bytes > 0 ? rows_bytes : 1);
     if (g < 1) g = 1;
     if (g > m2) g = m2;
     const int64_t groups = (m2 + g - 1) / g;
