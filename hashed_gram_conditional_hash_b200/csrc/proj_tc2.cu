@@ -47,7 +47,7 @@
 // loads are used anywhere (only the commit arrives on both CTAs' barriers).
 //
 // Tiles run over a persistent grid of as many pairs as fit, in groups of
-// M-blocks whose rows of e fill about 16 MB, N-tile by N-tile within a group:
+// M-blocks whose rows of e fill about 32 MB, N-tile by N-tile within a group:
 // a weight tile then serves the group's M-blocks while it is in L2, and the
 // group's rows of e stay in L2 for all its N-tiles (M-block-major order, all
 // N-tiles of one M-block before the next, re-read the weights from HBM once
@@ -69,10 +69,13 @@ namespace {
 using namespace tc;
 
 constexpr int kBM = 128;                    // token rows per CTA (pair: 256)
-// rows of e per group of M-blocks in the tile order (measured on the
-// HBM-scale workload, ms per step: 16 MB 4.66, 32 MB 4.72, 64 MB 5.11;
-// M-block by M-block 5.38 on another box against 5.02 for 32 MB)
-constexpr int64_t kTileGroupBytes = static_cast<int64_t>(16) << 20;
+// rows of e per group of M-blocks in the tile order.  Measured on the
+// HBM-scale workload (ms per step, DRAM reads per launch): M-block by M-block
+// 5.38 (8.76 GB) against 5.02 for 32 MB groups on one box; 16 MB 4.66, 32 MB
+// 4.72, 64 MB 5.11 on another with e and the weights at the same L2
+// priority; with e evict-last and the hidden state evict-first, 16 MB 4.75
+// (3.78 GB), 32 MB 4.72 (3.66 GB), 64 MB 5.02 (7.37 GB)
+constexpr int64_t kTileGroupBytes = static_cast<int64_t>(32) << 20;
 constexpr int kBN = 256;                    // output columns per pair tile
 constexpr int kBNh = kBN / 2;               // weight rows per CTA
 constexpr int kBK = 64;
@@ -267,9 +270,11 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_vo)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_vh)) : "memory");
     }
+    // the group's rows of e are read by every N-tile of the group: kept in L2
+    // before the weight tiles, which serve only the group's M-blocks in a row
     uint64_t pol_w, pol_a;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_w));
-    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol_a));
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol_w));
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_a));
     int stage = 0;
     uint32_t phase = 0;
     uint32_t pending = 0, pend_par = 0;      // stages armed by the leader (drain on abort)
@@ -368,12 +373,14 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
     uint32_t acc_phase = 0;
     const uint16_t* nk = static_cast<const uint16_t*>(p.norm_key);
     const uint16_t* nq = static_cast<const uint16_t*>(p.norm_query);
+    uint64_t pol_q;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol_q));
     // this warp's hidden-state slice, 64 columns at a time: {column, branch, token}
     auto fill_q = [&](int col, int h, int32_t tok) {
       if (lane == 0) {
         bulk_wait_group_read0();             // a V store from this tile has left it
         mbar_arrive_expect_tx(qbar, kXBytes);
-        tma_load_3d(xb, &map_q, col, h, tok, qbar);
+        tma_load_3d_hint(xb, &map_q, col, h, tok, qbar, pol_q);   // read once: evict first
       }
       q_inflight = true;
     };
@@ -661,6 +668,7 @@ cudaError_t launch_proj_tc2(const ProjParams& p, cudaStream_t s) {
     if (tp.n_split <= tp.nv_tiles * g_last) tp.group_mb = static_cast<int32_t>(g);
   }
   tp.force_timeout = (p.debug & ENGRAM_DEBUG_FORCE_TIMEOUT) ? 1 : 0;
+
   tp.timeout_ns = tp.force_timeout ? 20000000ull : 2000000000ull;
   // two K-blocks per TMA box when the head count allows it
   if (p.nh % 2 == 0) return launch_kc<2>(tp, p, s);
