@@ -44,3 +44,20 @@ def test_pass_roofline_large_workloads(name, tokens, total_bytes, total_flops):
     assert r["bytes_per_step"] == pytest.approx(total_bytes, rel=1e-3)
     assert r["flops_per_step"] == pytest.approx(total_flops, rel=1e-3)
     assert r["bound"] == "tensor"
+
+
+def test_device_memory_report_counts_every_buffer():
+    # one replica's device memory as the bench reports it: tables, weights,
+    # this step's inputs and output, the workspace, and the static scratch
+    import torch
+    from hashed_gram_conditional_hash_b200 import _lib as L
+    w = W.small_workload(B=2, T=16, hidden=256, hc_mult=2)
+    p = W.make_params(w, "cpu")
+    ws = torch.empty(4096, dtype=torch.uint8)
+    y = torch.empty((w.B, w.T, w.hc_mult, w.hidden), dtype=w.torch_dtype)
+    m = bench.device_memory(w, p, ws, y)
+    nb = lambda t: t.numel() * t.element_size()
+    assert m["tables"] == round(nb(p.table) / 1e9, 3)
+    assert m["inputs_outputs"] == round((nb(p.ids) + nb(p.hidden) + nb(y)) / 1e9, 3)
+    assert m["static_scratch"] == round(L.NO_ALLOC_SCRATCH_BYTES / 1e9, 3) == 0.034
+    assert set(m) == {"tables", "weights", "inputs_outputs", "workspace", "static_scratch"}
