@@ -724,6 +724,41 @@ def hbm_rates(device):
     return res
 
 
+def gemm_ref(args, w, device):
+    """cuBLAS (torch.matmul) on the projection's own GEMM shape, without its
+    epilogue: e [M, E] times the stacked value and key weights [E, H (1 + hc)],
+    bf16 in, fp32 accumulate, bf16 out.  Same L2 protocol as the timed steps
+    (flush and drain between launches); median of the launches by CUDA events.
+    It is the practical tensor-core rate for this shape on this GPU, beside
+    which the fused projection's rate can be read."""
+    M = w.B * (1 if w.decode_calls else w.T)
+    E = w.E
+    N = w.hidden * (1 + w.hc_mult)
+    g = torch.Generator(device=device).manual_seed(7)
+    a = (torch.randn(M, E, device=device, generator=g) * 0.5).to(torch.bfloat16)
+    b = (torch.randn(N, E, device=device, generator=g) * (E ** -0.5)).to(torch.bfloat16)
+    c = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+    flush = L2Flush(device)
+    n = max(5, min(args.steps, 50))
+    for i in range(3):
+        torch.matmul(a, b.t(), out=c)
+        flush(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i, (e0, e1) in enumerate(ev):
+        e0.record()
+        torch.matmul(a, b.t(), out=c)
+        e1.record()
+        flush(i)
+    torch.cuda.synchronize()
+    ms = sorted(x.elapsed_time(y) for x, y in ev)[n // 2]
+    flops = 2.0 * M * E * N
+    del a, b, c
+    return {"M": M, "K": E, "N": N, "launches": n, "median_us": ms * 1e3,
+            "tflops": flops / (ms / 1e3) / 1e12,
+            "note": "torch.matmul (cuBLAS) bf16, no epilogue, L2 flushed between launches"}
+
+
 def run_reference(args):
     """The reference arm: the float64 oracle on the host cores, K timed steps
     of a bounded sample each, sized so that warm-up + steps take ~2 minutes."""
@@ -778,6 +813,8 @@ def main():
                     help="also measure tables resident in pinned host memory (prefill workloads)")
     ap.add_argument("--hbm-rates", action="store_true",
                     help="also measure HBM write-only, read-only and copy rates (1 GiB torch kernels)")
+    ap.add_argument("--gemm-ref", action="store_true",
+                    help="also time cuBLAS on the projection's GEMM shape (no epilogue), for context")
     ap.add_argument("--sharded", type=int, default=0,
                     help="also time the device steps of a gather from a table sharded over this many GPUs")
     args = ap.parse_args()
@@ -805,6 +842,10 @@ def main():
             res["offload"] = run_offload(args, layer, p, w, device)
         if args.hbm_rates:
             res["hbm_rates"] = hbm_rates(device)
+        if args.gemm_ref:
+            res["gemm_ref"] = gemm_ref(args, w, device)
+            res["gemm_ref"]["projection_over_cublas"] = \
+                res["roofline"]["achieved"] / res["gemm_ref"]["tflops"]
         if args.sharded and not w.decode_calls:
             res["sharded"] = run_sharded(args, layer, p, w, device)
         from hashed_gram_conditional_hash_b200 import workloads as W

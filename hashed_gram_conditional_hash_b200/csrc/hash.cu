@@ -503,6 +503,9 @@ cudaError_t launch_hash(const HashParams& p, cudaStream_t s) {
   return cudaSuccess;
 }
 
+// Rows (token x head) up to which the 32-byte-row gather runs 128-thread blocks.
+constexpr int64_t kSmallGatherItems = int64_t{1} << 18;
+
 cudaError_t launch_hash_gather(const HashGatherParams& g0, cudaStream_t s) {
   HashGatherParams g = g0;
   const HashParams& p = g.h;
@@ -514,8 +517,12 @@ cudaError_t launch_hash_gather(const HashGatherParams& g0, cudaStream_t s) {
     constexpr int kRows = 16;                    // rows per warp for 128-byte rows
     if (total * (32 / kRows) + 256 > INT32_MAX) return cudaErrorInvalidValue;  // 32-bit ids in the kernel
     if (w32_form(g)) {
-      const int64_t blocks = (total + 255) / 256;
-      launch_k(hash_gather_w32_kernel<1>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, g);
+      // A launch of at most a few waves spreads more evenly over the SMs in
+      // 128-thread blocks (model-shaped and decode batches: 0.3-0.5 us less per
+      // step); a large one keeps 256 (0.9 % faster on the 17 GB table).
+      const int bt = total <= kSmallGatherItems ? 128 : 256;
+      const int64_t blocks = (total + bt - 1) / bt;
+      launch_k(hash_gather_w32_kernel<1>, dim3(static_cast<unsigned>(blocks)), dim3(bt), 0, s, g);
     } else if (g.row_bytes == 128) {
       const int64_t blocks = (total + 8 * kRows - 1) / (8 * kRows);
       if (g.table_host)
