@@ -92,7 +92,7 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, smax, reasons = [], [], set()
+        sm, smax, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
@@ -104,6 +104,10 @@ class ClockSampler:
                     smax.append(float(parts[3]))
                 except ValueError:
                     continue
+                try:
+                    pw.append(float(parts[4]))
+                except ValueError:
+                    pass
                 for n, v in zip(names, parts[6:10]):
                     if v.lower() == "active":
                         reasons.add(n)
@@ -111,6 +115,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax),
+                "power_w": float(np.median(pw)) if pw else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
