@@ -373,6 +373,8 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
     uint32_t acc_phase = 0;
     const uint16_t* nk = static_cast<const uint16_t*>(p.norm_key);
     const uint16_t* nq = static_cast<const uint16_t*>(p.norm_query);
+    // hidden-state slices are read once, V tiles and score partials are read
+    // by later kernels: none of them should displace the operand tiles in L2
     uint64_t pol_q;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol_q));
     // this warp's hidden-state slice, 64 columns at a time: {column, branch, token}
@@ -420,7 +422,7 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
           fence_proxy_async();  // the tile's generic writes are visible to the tensor store
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&map_vo, xb, cc + f * kXCols, static_cast<int32_t>(tok0));
+            tma_store_2d_hint(&map_vo, xb, cc + f * kXCols, static_cast<int32_t>(tok0), pol_q);
             bulk_commit_group();
           }
         }
@@ -480,7 +482,8 @@ proj_tc2_kernel(const __grid_constant__ Tc2Params tp, const __grid_constant__ CU
         }
         const float dot = dot2.x + dot2.y, ssk = ssk2.x + ssk2.y, ssq = ssq2.x + ssq2.y;
         if (fine && live)
-          p.partials[(m * p.hc + h) * p.n_tiles + cc / kEpiCols] = make_float4(dot, ssk, ssq, 0.f);
+          st_global_v4_hint(p.partials + (m * p.hc + h) * p.n_tiles + cc / kEpiCols, make_float4(dot, ssk, ssq, 0.f),
+                            pol_q);
       }
       if (!fine) break;
       // the warp's TMEM reads are complete (tcgen05.wait::ld) before lane 0
