@@ -497,9 +497,50 @@ def run_e2e(args, layer, p, w, device, world):
     ms = max_over_ranks(t, world).item()
     h2d = ids_h.numel() * 8 + hid_h.numel() * hid_h.element_size()
     d2h = y_h[0].numel() * y_h[0].element_size()
-    return {"value": job_throughput(world, Bq * Tq, K, ms), "unit": "tokens/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "overlap": "copies of neighbouring steps overlap the forward (3 streams, 2 buffers)"}
+    value = job_throughput(world, Bq * Tq, K, ms)
+    res = {"value": value, "unit": "tokens/s",
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+           "overlap": "copies of neighbouring steps overlap the forward (3 streams, 2 buffers)"}
+    link = host_link_rates(hid_h, hid_d[0], y_h[0], y_d[0], s_in, s_out)
+    # with the copies of neighbouring steps overlapped, a step can go no faster
+    # than its slower direction at the rates both directions reach together
+    bound_s = max(h2d / (link["h2d_concurrent_gbs"] * 1e9), d2h / (link["d2h_concurrent_gbs"] * 1e9))
+    link["bound_tokens_per_s"] = world * Bq * Tq / bound_s
+    link["frac"] = value / link["bound_tokens_per_s"]
+    res["host_link"] = link
+    return res
+
+
+def host_link_rates(src_h, dst_d, dst_h, src_d, s_in, s_out):
+    """Pinned host <-> device copy rates with the step's own buffers: each
+    direction alone, then both at once on two streams (median of 3, CUDA
+    events on the copying streams)."""
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+
+    def timed(pairs):
+        out = []
+        for _ in range(3):
+            ev = []
+            torch.cuda.synchronize()
+            for stream, dst, src in pairs:
+                a, b = mk(), mk()
+                a.record(stream)
+                with torch.cuda.stream(stream):
+                    dst.copy_(src, non_blocking=True)
+                b.record(stream)
+                ev.append((a, b))
+            torch.cuda.synchronize()
+            out.append([a.elapsed_time(b) for a, b in ev])
+        return [sorted(x[i] for x in out)[1] for i in range(len(pairs))]
+
+    nb_in = src_h.numel() * src_h.element_size()
+    nb_out = src_d.numel() * src_d.element_size()
+    (t_in,) = timed([(s_in, dst_d, src_h)])
+    (t_out,) = timed([(s_out, dst_h, src_d)])
+    t_in2, t_out2 = timed([(s_in, dst_d, src_h), (s_out, dst_h, src_d)])
+    return {"h2d_gbs": nb_in / t_in / 1e6, "d2h_gbs": nb_out / t_out / 1e6,
+            "h2d_concurrent_gbs": nb_in / t_in2 / 1e6, "d2h_concurrent_gbs": nb_out / t_out2 / 1e6,
+            "bytes": [int(nb_in), int(nb_out)]}
 
 
 def run_offload(args, layer, p, w, device):
