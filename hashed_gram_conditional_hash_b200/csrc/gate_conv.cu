@@ -416,7 +416,7 @@ constexpr int kTileTMin = 32;     // positions per block: the launcher picks one
 constexpr int kTileTMax = 64;     // [32, 64] that spreads the blocks evenly over the SMs
 constexpr int kTileC = 256;       // channels per block (512 bytes of a bf16 row)
 constexpr int kTileMaxDil = 32;   // longer halos take the run form
-constexpr int kStepSeq = 4;       // sequences per block of the decode step
+constexpr int kStepSeq = 8;       // sequences per block of the decode step
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -653,96 +653,114 @@ __global__ void __launch_bounds__(kSlimThreads, 6) conv_slim_kernel(const __grid
 }
 
 // One decode step (T = 1) with the streaming state, K = 4 taps, bfloat16:
-// block (group of kStepSeq sequences, 256-channel slice), one warp per
-// branch, 8 channels per lane.  Before its programmatic-launch wait (the
-// gate kernel lets this grid start early) a lane loads its taps once for the
-// group, every sequence's pos (advanced by this call's hash kernel), turns
-// pos into the ring rows of the taps at t - 3 dil, t - 2 dil, t - dil (the
-// ring holds (K-1) dil + 1 >= 3 dil + 1 positions, slot = position mod ring
-// length, by invariant-divisor multiplication) and loads its pieces of those
-// rows and their gates, all written by earlier calls; after the wait, its
-// 16-byte piece of V(t) and the step's gate; then it stores 8 channels of Y
-// per sequence.  No block barrier.  The same kernel is the step's state
+// block (group of S sequences, 256-channel slice), one warp per branch, 8
+// channels per lane.  What the branch warps share is staged once per block
+// in shared memory by cp.async, so no thread holds loads in registers across
+// the wait and the whole decode batch fits in one wave of blocks.  Before its
+// programmatic-launch wait (the gate kernel lets this grid start early) the
+// block reads each sequence's pos (advanced by this call's hash kernel),
+// turns it into the ring rows of the taps at t - 3 dil, t - 2 dil, t - dil
+// (the ring holds (K-1) dil + 1 >= 3 dil + 1 positions, slot = position mod
+// ring length, by invariant-divisor multiplication) and copies those rows'
+// slices and gates, all written by earlier calls; after the wait, V(t) and
+// g(t).  Each branch warp then forms U = g V of the four rows from shared
+// memory and stores 8 channels of Y per lane and sequence, in the same order
+// of operations as the prefill forms.  The same kernel is the step's state
 // advance: the branch-0 warp writes V(t) and lanes 0 write g(t) into t's
 // slot, which no tap of this step reads.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+
 template <int S>
-__global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __grid_constant__ ConvParams p) {
+__global__ void __launch_bounds__(32 * ENGRAM_MAX_HC, 4) conv_step_kernel(const __grid_constant__ ConvParams p) {
   constexpr int K = 4;
+  constexpr int kPieces = kTileC * 2 / 16;          // 16-byte pieces of a row's slice
+  __shared__ __align__(16) uint16_t s_rows[S][K][kTileC];   // taps' rows, then V(t)
+  __shared__ float s_g[S][K][ENGRAM_MAX_HC];
+  __shared__ int64_t s_ring[S][K];                 // ring row of each tap (-1: zeros); [K-1]: t's slot
   const int tid = static_cast<int>(threadIdx.x);
+  const int nthr = static_cast<int>(blockDim.x);
   const int h = tid >> 5, lane = tid & 31;
-  if (h >= p.hc) return;
   const int b0 = static_cast<int>(blockIdx.x) * S;
-  const int c = static_cast<int>(blockIdx.y) * kTileC + lane * 8;
+  const int c0 = static_cast<int>(blockIdx.y) * kTileC;
+  const int c = c0 + lane * 8;
   const uint16_t* V = static_cast<const uint16_t*>(p.V);
   uint16_t* vr = static_cast<uint16_t*>(const_cast<void*>(p.v_ring));
   float* gr = const_cast<float*>(p.g_ring);
-  uint4 raw[S][K];
-  float gg[S][K];
-  // Before the wait: what no kernel of this call after the hash writes.  pos
-  // was advanced by this call's hash kernel (finished before the projection
-  // began), the ring rows of the taps by earlier calls, the taps are
-  // weights; the gate kernel lets this grid start while it runs, so these
-  // dependent loads (pos, then the rows it selects) overlap the gates.
-  // Read through L2 (the state is written by other grids).
-  int64_t P[S];
-  int64_t row_t[S];
-#pragma unroll
-  for (int s = 0; s < S; ++s) P[s] = (b0 + s < p.B) ? __ldcg(p.pos + b0 + s) - p.pos_lag : -1;
-  float2 w2[4][K];                                // [channel pair][tap]
-  {
-    float w[8][K];
-    load_taps<uint16_t, K>(static_cast<const uint16_t*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, K, w);
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int i = 0; i < K; ++i) w2[j][i] = make_float2(w[2 * j][i], w[2 * j + 1][i]);
-  }
-#pragma unroll
-  for (int s = 0; s < S; ++s) {
-    const int64_t Ps = P[s];                        // position of this step's token (-1: no sequence)
+  const uint32_t s_rows0 = static_cast<uint32_t>(__cvta_generic_to_shared(&s_rows[0][0][0]));
+  const uint32_t s_g0 = static_cast<uint32_t>(__cvta_generic_to_shared(&s_g[0][0][0]));
+
+  // (1) before the wait: the taps' ring rows, from pos (through L2: another
+  // grid wrote it), and this lane's conv taps (weights)
+  if (tid < S) {
+    const int b = b0 + tid;
+    const int64_t Ps = b < p.B ? __ldcg(p.pos + b) - p.pos_lag : -1;   // position of t (-1: no sequence)
     const int64_t slot_t = (Ps >= 0 && Ps < INT32_MAX)
                                ? static_cast<int64_t>(Ps - static_cast<int64_t>(fast_div(static_cast<uint32_t>(Ps), p.div_ring)) *
                                                               p.ring_len)
                                : (Ps >= 0 ? Ps % p.ring_len : 0);
-    const int64_t ring0 = static_cast<int64_t>(b0 + s) * p.ring_len;
-    row_t[s] = ring0 + slot_t;
+    const int64_t ring0 = static_cast<int64_t>(b) * p.ring_len;
 #pragma unroll
     for (int i = 0; i < K - 1; ++i) {               // tap i sits at t - (K-1-i) dil
       const int64_t back = static_cast<int64_t>(K - 1 - i) * p.dil;
       int64_t slot = slot_t - back;
       if (slot < 0) slot += p.ring_len;
-      if (Ps - back >= 0) {                         // also false past the last sequence (P = -1)
-        const int64_t row = ring0 + slot;
-        raw[s][i] = __ldcg(reinterpret_cast<const uint4*>(vr + row * p.H + c));
-        gg[s][i] = __ldcg(gr + row * p.hc + h);
-      } else {
-        raw[s][i] = make_uint4(0, 0, 0, 0);
-        gg[s][i] = 0.f;
-      }
+      s_ring[tid][i] = (Ps - back >= 0) ? ring0 + slot : -1;   // also -1 past the last sequence
     }
+    s_ring[tid][K - 1] = b < p.B ? ring0 + slot_t : -1;
   }
+  float2 w2[4][K];                                // [channel pair][tap]
+  if (h < p.hc)
+    load_taps_pairs<8>(static_cast<const uint16_t*>(p.conv_w) + (static_cast<int64_t>(h) * p.H + c) * K, w2);
+  __syncthreads();
+  for (int i = tid; i < S * (K - 1) * kPieces; i += nthr) {
+    const int sq = i / ((K - 1) * kPieces), r = (i / kPieces) % (K - 1), k = i % kPieces;
+    const uint32_t dst = s_rows0 + static_cast<uint32_t>(((sq * K + r) * kTileC + k * 8) * 2);
+    const int64_t row = s_ring[sq][r];
+    if (row >= 0) cp_async16(dst, vr + row * p.H + c0 + k * 8);
+    else asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+  }
+  for (int i = tid; i < S * (K - 1) * p.hc; i += nthr) {
+    const int sq = i / ((K - 1) * p.hc), r = (i / p.hc) % (K - 1), hh = i % p.hc;
+    const int64_t row = s_ring[sq][r];
+    if (row >= 0) cp_async4(s_g0 + static_cast<uint32_t>(((sq * K + r) * ENGRAM_MAX_HC + hh) * 4), gr + row * p.hc + hh);
+    else s_g[sq][r][hh] = 0.f;
+  }
+
   pdl_wait();  // the gate kernel (and so the projection) has finished: V(t), g(t)
-#pragma unroll
-  for (int s = 0; s < S; ++s) {
-    const int b = b0 + s;
-    if (b < p.B) {
-      raw[s][K - 1] = __ldg(reinterpret_cast<const uint4*>(V + static_cast<int64_t>(b) * p.H + c));
-      gg[s][K - 1] = __ldg(p.g + static_cast<int64_t>(b) * p.hc + h);
-    } else {
-      raw[s][K - 1] = make_uint4(0, 0, 0, 0);
-      gg[s][K - 1] = 0.f;
-    }
+  for (int i = tid; i < S * kPieces; i += nthr) {
+    const int sq = i / kPieces, k = i % kPieces;
+    const int b = b0 + sq;
+    const uint32_t dst = s_rows0 + static_cast<uint32_t>(((sq * K + K - 1) * kTileC + k * 8) * 2);
+    if (b < p.B) cp_async16(dst, V + static_cast<int64_t>(b) * p.H + c0 + k * 8);
+    else asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
   }
-#pragma unroll
-  for (int s = 0; s < S; ++s) {
-    const int b = b0 + s;
+  for (int i = tid; i < S * p.hc; i += nthr) {
+    const int sq = i / p.hc, hh = i - sq * p.hc;
+    const int b = b0 + sq;
+    if (b < p.B) cp_async4(s_g0 + static_cast<uint32_t>(((sq * K + K - 1) * ENGRAM_MAX_HC + hh) * 4),
+                           p.g + static_cast<int64_t>(b) * p.hc + hh);
+    else s_g[sq][K - 1][hh] = 0.f;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  if (h >= p.hc) return;
+
+  // (2) outputs and the state advance
+  for (int sq = 0; sq < S; ++sq) {
+    const int b = b0 + sq;
     if (b >= p.B) break;
     float2 u[K][4];
+    uint4 vt;
 #pragma unroll
     for (int i = 0; i < K; ++i) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(&s_rows[sq][i][lane * 8]);
+      if (i == K - 1) vt = raw;
       float2 v[4];
-      Pair8<uint16_t>::unpack(raw[s][i], v);
-      const float2 g2 = make_float2(gg[s][i], gg[s][i]);
+      Pair8<uint16_t>::unpack(raw, v);
+      const float gg = s_g[sq][i][h];
+      const float2 g2 = make_float2(gg, gg);
 #pragma unroll
       for (int j = 0; j < 4; ++j) u[i][j] = __fmul2_rn(g2, v[j]);
     }
@@ -755,9 +773,9 @@ __global__ void __launch_bounds__(32 * ENGRAM_MAX_HC) conv_step_kernel(const __g
       acc[j] = a;
     }
     Pair8<uint16_t>::store(static_cast<uint16_t*>(p.Y) + (static_cast<int64_t>(b) * p.hc + h) * p.H + c, acc);
-    // the step's state advance
-    if (h == 0) *reinterpret_cast<uint4*>(vr + row_t[s] * p.H + c) = raw[s][K - 1];
-    if (blockIdx.y == 0 && lane == 0) gr[row_t[s] * p.hc + h] = gg[s][K - 1];
+    const int64_t row_t = s_ring[sq][K - 1];
+    if (h == 0) *reinterpret_cast<uint4*>(vr + row_t * p.H + c) = vt;
+    if (blockIdx.y == 0 && lane == 0) gr[row_t * p.hc + h] = s_g[sq][K - 1][h];
   }
 }
 
