@@ -713,7 +713,7 @@ PROBE_OPS = {"write_v4": 0, "write_v8": 1, "write_v4_cs": 2, "write_bulk": 3, "r
              "copy_v4": 6, "copy_v8": 7}
 
 
-def hbm_rates(device):
+def hbm_rates(device, table=None, n_rows=0):
     """HBM write-only, read-only and copy rates on 1 GiB buffers: this
     library's probe kernels (16- and 32-byte stores and loads, evict-first
     stores, bulk-copy-engine stores; libengram_probe.so) beside torch's fill,
@@ -764,6 +764,30 @@ def hbm_rates(device):
                 best = (rate, blocks)
         res[name + "_gbs"] = best[0]
         res[name + "_blocks"] = best[1]
+    if table is not None and n_rows > 0:
+        # random 128-byte rows out of the workload's own table, as many as one
+        # step gathers: the access pattern of the hash+gather stage without
+        # its hash (read + write bytes over time)
+        lib.engram_probe_gather.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_size_t,
+                                            ctypes.c_int, ctypes.c_void_p]
+        out = torch.empty(n_rows * 128, dtype=torch.uint8, device=device)
+        src_bytes = (table.numel() * table.element_size()) // 128 * 128
+        best = None
+        for blocks_per_sm in (4, 8, 16):
+            blocks = blocks_per_sm * torch.cuda.get_device_properties(device).multi_processor_count
+
+            def run():
+                rc = lib.engram_probe_gather(out.data_ptr(), table.data_ptr(), out.numel(), src_bytes, blocks,
+                                             stream.cuda_stream)
+                if rc != 0:
+                    raise RuntimeError("gather probe failed: %d" % rc)
+            ms = med_ms(run)
+            rate = 2 * out.numel() / ms / 1e6
+            if best is None or rate > best[0]:
+                best = (rate, blocks)
+        res["gather_random_rows_gbs"], res["gather_random_rows_blocks"] = best
+        res["gather_random_rows"] = {"rows": int(n_rows), "table_bytes": int(src_bytes)}
+        del out
     res["write_only_gbs"] = max(res[k + "_gbs"] for k in ("write_v4", "write_v8", "write_v4_cs", "write_bulk"))
     res["read_only_gbs"] = max(res["read_v4_gbs"], res["read_v8_gbs"])
     res["copy_gbs"] = max(res["copy_v4_gbs"], res["copy_v8_gbs"])
@@ -887,7 +911,8 @@ def main():
         if args.offload and not w.decode_calls:
             res["offload"] = run_offload(args, layer, p, w, device)
         if args.hbm_rates:
-            res["hbm_rates"] = hbm_rates(device)
+            tab = p.table if (p.table is not None and p.table.is_cuda and w.row_dim * p.table.element_size() == 128) else None
+            res["hbm_rates"] = hbm_rates(device, tab, w.M * w.nh)
         if args.gemm_ref:
             res["gemm_ref"] = gemm_ref(args, w, device)
             res["gemm_ref"]["projection_over_cublas"] = \

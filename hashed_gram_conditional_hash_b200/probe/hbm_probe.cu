@@ -11,6 +11,7 @@
 //   3 write, cp.async.bulk from a 32 KB shared tile (the bulk-copy engine)
 //   4 read, 16-byte ld.global.nc          5 read, 32-byte ld.global.nc.v8
 //   6 copy, 16-byte                        7 copy, 32-byte
+// and engram_probe_gather: random 128-byte rows out of a large source.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -109,7 +110,61 @@ __global__ void __launch_bounds__(32) bulk_write_kernel(char* dst, int64_t n_chu
   __syncwarp();
 }
 
+// Random-row gather: 128-byte rows at pseudo-random indices of a source of
+// n_src rows, written densely; a warp moves 32 rows as four 32-byte pieces
+// per lane, all loads before the first store (the access form of the
+// pass's hash+gather kernel, without the hash).
+__global__ void __launch_bounds__(256) gather_rows_kernel(char* dst, const char* src, int64_t n_rows,
+                                                          uint64_t n_src) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t q0 = warp * 32; q0 < n_rows; q0 += nwarps * 32) {
+    uint64_t x = static_cast<uint64_t>(q0 + lane) * 0x9E3779B97F4A7C15ull;
+    x ^= x >> 29;
+    const int64_t row = static_cast<int64_t>(x % n_src);
+    uint32_t r[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = u * 32 + lane;
+      const int64_t srow = __shfl_sync(0xffffffffu, row, i >> 2);
+      if (q0 + (i >> 2) < n_rows)
+        asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[u][0]), "=r"(r[u][1]), "=r"(r[u][2]), "=r"(r[u][3]), "=r"(r[u][4]), "=r"(r[u][5]),
+                       "=r"(r[u][6]), "=r"(r[u][7])
+                     : "l"(src + srow * 128 + (i & 3) * 32));
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = u * 32 + lane;
+      if (q0 + (i >> 2) < n_rows)
+        asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst + q0 * 128 + i * 32),
+                     "r"(r[u][0]), "r"(r[u][1]), "r"(r[u][2]), "r"(r[u][3]), "r"(r[u][4]), "r"(r[u][5]),
+                     "r"(r[u][6]), "r"(r[u][7])
+                     : "memory");
+    }
+  }
+}
+
 }  // namespace
+
+// Gathers out_bytes / 128 rows of 128 bytes from a source of src_bytes (both
+// multiples of 128, pointers 32-byte aligned) at pseudo-random row indices;
+// blocks = grid size (<= 0: 8 per SM).  Returns a cudaError_t.
+extern "C" int engram_probe_gather(void* dst, const void* src, size_t out_bytes, size_t src_bytes, int blocks,
+                                   void* stream) {
+  if (out_bytes % 128 != 0 || src_bytes % 128 != 0 || src_bytes == 0 ||
+      (reinterpret_cast<uintptr_t>(dst) & 31u) != 0 || (reinterpret_cast<uintptr_t>(src) & 31u) != 0)
+    return static_cast<int>(cudaErrorInvalidValue);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (blocks <= 0) blocks = 8 * sms;
+  gather_rows_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<char*>(dst), static_cast<const char*>(src), static_cast<int64_t>(out_bytes / 128),
+      static_cast<uint64_t>(src_bytes / 128));
+  return static_cast<int>(cudaGetLastError());
+}
 
 // Runs op once on the stream; blocks = grid size (<= 0: 4 per SM).  Returns a
 // cudaError_t.
