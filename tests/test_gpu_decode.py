@@ -28,7 +28,9 @@ def _decode_all(layer, ids_bt, hidden_tb):
     steps = ids_bt.t().contiguous().view(S, B, 1)
     ys = torch.empty((S, B, 1, layer.hc, layer.hidden), dtype=layer.dtype, device=DEV)
     for c in range(S):
-        layer.forward(steps[c], hidden_tb[c].view(B, 1, layer.hc, layer.hidden), y=ys[c],
+        # each step's ids in a buffer of their own: the ABI takes 16-byte aligned
+        # pointers, and a row of the [S, B] view starts at c * B * 8 bytes
+        layer.forward(steps[c].clone(), hidden_tb[c].view(B, 1, layer.hc, layer.hidden), y=ys[c],
                       ws=ws, state=state, dev_status=st)
     assert L.engram_read_status(st) == 0
     assert torch.all(state.pos == S)
@@ -77,6 +79,25 @@ def test_chunked_prefill_with_state(chunks):
     # the chunks together are the oracle's prefill over the whole sequence
     ref = oracle_forward_full(p)
     assert rel_err(y.double().cpu().numpy(), ref["Y"]) <= TOL[w.dtype]
+
+
+@pytest.mark.parametrize("B,hc,hidden,dil,orders", [(9, 1, 512, 3, (2, 3)), (17, 4, 768, 2, (2,)),
+                                                     (8, 3, 256, 5, (2, 3, 5))])
+def test_decode_steps_partial_blocks_and_branch_counts(B, hc, hidden, dil, orders):
+    # every token a decode step (T = 1 with the state): batches that leave the
+    # decode conv's last block of sequences partly empty, one to four branches,
+    # several 256-channel slices, dilations whose ring wraps several times
+    T = 40
+    w = W.small_workload(B=B, T=T, orders=orders, dilation=dil, hidden=hidden, hc_mult=hc)
+    p = device_params(w)
+    layer = EngramLayer.from_params(p)
+    ys, state = _decode_all(layer, p.ids, p.hidden.transpose(0, 1).contiguous())
+    y = ys.transpose(0, 1)                                  # [B, T, hc, H]
+    y_pre = layer.forward(p.ids, p.hidden)
+    err = (y.double() - y_pre.double()).abs().max().item()
+    assert err <= 1e-2 * y_pre.double().abs().max().item()
+    assert rel_err(y.double().cpu().numpy(), oracle_forward_full(p)["Y"]) <= TOL[w.dtype]
+    assert torch.all(state.pos == T)
 
 
 def test_streaming_with_raw_ids_keeps_compressed_ids_in_the_ring():
