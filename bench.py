@@ -47,12 +47,24 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 def load_peaks():
+    """Peaks from MEASURED_PEAKS.json when it holds them (numbers under the
+    keys of PEAKS_FALLBACK), else the machine's fallback figures, key by key."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return d, "measured"
-    except OSError:
-        return PEAKS_FALLBACK, "fallback"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+    peaks, measured = dict(PEAKS_FALLBACK), []
+    for k in PEAKS_FALLBACK:
+        v = d.get(k) if isinstance(d, dict) else None
+        if isinstance(v, (int, float)) and v > 0:
+            peaks[k] = float(v)
+            measured.append(k)
+    if len(measured) == len(PEAKS_FALLBACK):
+        return peaks, "measured"
+    if not measured:
+        return peaks, "fallback"
+    return peaks, "measured (%s), else fallback" % ", ".join(measured)
 
 
 # ---------------------------------------------------------------- clocks

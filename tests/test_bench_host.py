@@ -61,3 +61,23 @@ def test_device_memory_report_counts_every_buffer():
     assert m["inputs_outputs"] == round((nb(p.ids) + nb(p.hidden) + nb(y)) / 1e9, 3)
     assert m["static_scratch"] == round(L.NO_ALLOC_SCRATCH_BYTES / 1e9, 3) == 0.034
     assert set(m) == {"tables", "weights", "inputs_outputs", "workspace", "static_scratch"}
+
+
+def test_load_peaks_takes_measured_figures_key_by_key(tmp_path, monkeypatch):
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, kind = bench.load_peaks()                       # no file: the fallback figures
+    assert kind == "fallback" and peaks == bench.PEAKS_FALLBACK
+    f = tmp_path / "MEASURED_PEAKS.json"
+    f.write_text(json.dumps({"hbm_gbs": 6550.4, "bf16_tflops": 1661.2, "bf16_tflops_sustained": 1396.1,
+                             "clocks": {"sm_mhz": 1965}}))
+    peaks, kind = bench.load_peaks()
+    assert kind == "measured"
+    assert peaks == {"hbm_gbs": 6550.4, "bf16_tflops": 1661.2, "bf16_tflops_sustained": 1396.1}
+    f.write_text(json.dumps({"hbm_gbs": 6550.4, "bf16_tflops": "n/a"}))   # partial: the rest falls back
+    peaks, kind = bench.load_peaks()
+    assert peaks["hbm_gbs"] == 6550.4
+    assert peaks["bf16_tflops"] == bench.PEAKS_FALLBACK["bf16_tflops"]
+    assert kind.startswith("measured (hbm_gbs)")
+    f.write_text("not json")
+    assert bench.load_peaks() == (bench.PEAKS_FALLBACK, "fallback")
