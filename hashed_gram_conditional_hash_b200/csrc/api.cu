@@ -101,6 +101,17 @@ engram_status check_config(const engram_config* c) {
 }
 
 // Shapes the projection, gate and conv kernels need.
+// The kernels index (token, head) rows with 32-bit integers (the 16-rows-per-
+// warp gather needs 2 rows + 256 < 2^31): a call hashes and gathers at most
+// 2^30 rows, B*T*heads.
+engram_status check_row_count(const engram_config* cfg, int32_t B, int32_t T) {
+  const int64_t rows = static_cast<int64_t>(B) * T * cfg->n_orders * cfg->heads_per_order;
+  if (rows > (int64_t{1} << 30))
+    return fail(ENGRAM_ERR_UNSUPPORTED, "B*T*heads = %lld rows exceeds 2^30 per call; split the batch",
+                static_cast<long long>(rows));
+  return ENGRAM_OK;
+}
+
 engram_status check_dense_shapes(const engram_config* c) {
   if (c->hidden % 64 != 0)
     return fail(ENGRAM_ERR_UNSUPPORTED, "hidden=%d must be a multiple of 64", c->hidden);
@@ -225,6 +236,10 @@ engram_status prepare_gather(const engram_config* cfg, const engram_weights* wts
                              int32_t B, int32_t T, const int64_t* history, void* e, uint32_t* dev_status,
                              HashGatherParams* hg, bool with_table = true) {
   if (wts == nullptr) return fail(ENGRAM_ERR_INVALID_ARG, "weights is NULL");
+  {
+    const engram_status sr = check_row_count(cfg, B, T);
+    if (sr != ENGRAM_OK) return sr;
+  }
   const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
   if (row_bytes % 16 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
   if (ids == nullptr || !aligned16(ids)) return fail(ENGRAM_ERR_INVALID_ARG, "ids must be non-NULL, 16-byte aligned");
@@ -785,6 +800,8 @@ engram_status engram_forward(const engram_config* cfg, const engram_weights* wts
   if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
   const int64_t M = static_cast<int64_t>(B) * T;
   if (M == 0) return ENGRAM_OK;
+  st = check_row_count(cfg, B, T);
+  if (st != ENGRAM_OK) return st;
   const void* ptrs[] = {wts->table, wts->w_value, wts->w_key, wts->norm_key, wts->norm_query,
                         wts->conv_w, hidden, y, ws, ids};
   for (const void* p : ptrs) {
@@ -915,6 +932,8 @@ engram_status engram_forward_gathered(const engram_config* cfg, const engram_wei
   if (B < 0 || T < 0) return fail(ENGRAM_ERR_INVALID_ARG, "B, T must be >= 0");
   const int64_t M = static_cast<int64_t>(B) * T;
   if (M == 0) return ENGRAM_OK;
+  st = check_row_count(cfg, B, T);
+  if (st != ENGRAM_OK) return st;
   const int row_bytes = cfg->row_dim * (cfg->dtype == ENGRAM_F32 ? 4 : 2);
   if (row_bytes % 16 != 0) return fail(ENGRAM_ERR_UNSUPPORTED, "rows must be a multiple of 16 bytes");
   const void* ptrs[] = {e, wts->w_value, wts->w_key, wts->norm_key, wts->norm_query, wts->conv_w, hidden, y, ws};

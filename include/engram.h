@@ -277,7 +277,11 @@ engram_status engram_state_init(const engram_config* cfg, const engram_state* st
  *   ws:     DEVICE scratch of engram_forward_workspace_size(cfg, B, T) bytes,
  *           256-byte aligned.
  * Requirements: H % 64 == 0; bfloat16 with Dh == 64 and H % 256 == 0 runs the
- * tensor-core (tcgen05) projection, other shapes the CUDA-core one. */
+ * tensor-core (tcgen05) projection, other shapes the CUDA-core one.  At most
+ * 2^30 (token, head) rows per call: B*T*n_orders*heads_per_order above that
+ * returns ENGRAM_ERR_UNSUPPORTED before any launch (split the batch); this
+ * limit also holds for engram_gather_ids, engram_gather_ids_layers and
+ * engram_forward_gathered. */
 engram_status engram_forward(const engram_config* cfg, const engram_weights* weights,
                              const int64_t* ids, int32_t B, int32_t T, const void* hidden,
                              void* y, const engram_state* state, void* ws, size_t ws_bytes,

@@ -100,6 +100,28 @@ def test_forward_rejects_null_and_misaligned():
     assert rc == 1 and "aligned" in L.last_error()
 
 
+def test_row_count_above_2_30_is_unsupported_before_any_pointer_is_read():
+    # B*T*heads above 2^30: the kernels index (token, head) rows in 32 bits, so
+    # the forward, the gathers and the forward from gathered rows refuse the
+    # call on the host (the pointers below are never dereferenced)
+    cfg = _cfg()                                           # 2 orders x 2 heads
+    w = L.EngramWeights()
+    B, T = 1 << 14, 1 << 15                                 # 2^29 tokens x 4 heads = 2^31 rows
+    rc = L.lib().engram_forward(C.byref(cfg), C.byref(w), C.c_void_p(256), B, T, C.c_void_p(256),
+                                C.c_void_p(256), None, C.c_void_p(256), 0, None, None)
+    assert rc == 2 and "2^30" in L.last_error()
+    rc = L.lib().engram_gather_ids(C.byref(cfg), C.byref(w), C.c_void_p(256), B, T, None, C.c_void_p(256),
+                                   None, None)
+    assert rc == 2 and "2^30" in L.last_error()
+    rc = L.lib().engram_forward_gathered(C.byref(cfg), C.byref(w), C.c_void_p(256), B, T, C.c_void_p(256),
+                                         C.c_void_p(256), C.c_void_p(256), 0, None, None)
+    assert rc == 2 and "2^30" in L.last_error()
+    # 2^30 rows exactly is accepted by the count check (the null weights fail later)
+    rc = L.lib().engram_gather_ids(C.byref(cfg), C.byref(w), C.c_void_p(256), 1 << 14, 1 << 14, None,
+                                   C.c_void_p(256), None, None)
+    assert "2^30" not in L.last_error()
+
+
 def test_short_conv_rejects_aliasing():
     cfg = _cfg()
     rc = L.lib().engram_short_conv(C.byref(cfg), C.c_void_p(256), 1, 4, C.c_void_p(512), None,
