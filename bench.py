@@ -433,6 +433,8 @@ def run_ours(args, rank, world, device):
         "roofline": {"bound": "tensor", "kernel": kname,
                      "achieved": proj_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": proj_tflops / tc_peak, "peak_kind": "%s bf16 %s" % (peak_kind, "sustained" if sustained else "burst"),
+                     "frac_of_burst": proj_tflops / peaks["bf16_tflops"],
+                     "frac_of_sustained": proj_tflops / peaks["bf16_tflops_sustained"],
                      "traffic": kernel_traffic(kname, w.name),
                      "flops_per_launch": a["proj_flops"] * tokens_step},
         "pass_roofline": pass_roofline(w, tokens_step, t_step / K / 1e3, tc_peak, peaks["hbm_gbs"]),
