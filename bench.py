@@ -802,6 +802,19 @@ def hbm_rates(device, table=None, n_rows=0):
         res["gather_random_rows_gbs"], res["gather_random_rows_blocks"] = best
         res["gather_random_rows"] = {"rows": int(n_rows), "table_bytes": int(src_bytes)}
         del out
+    # fp32 multiply-add rate, packed pairs against scalar (16 independent chains
+    # per thread, 8 blocks of 256 per SM)
+    lib.engram_probe_fma.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    fblocks = 8 * torch.cuda.get_device_properties(device).multi_processor_count
+    fout = torch.empty(fblocks * 256, dtype=torch.float32, device=device)
+    iters = 4096
+    for name, packed in (("fma_packed_tflops", 1), ("fma_scalar_tflops", 0)):
+        def run():
+            rc = lib.engram_probe_fma(packed, fout.data_ptr(), fblocks, iters, stream.cuda_stream)
+            if rc != 0:
+                raise RuntimeError("fma probe failed: %d" % rc)
+        res[name] = 2.0 * 16 * iters * fblocks * 256 / med_ms(run) / 1e9
+    del fout
     res["write_only_gbs"] = max(res[k + "_gbs"] for k in ("write_v4", "write_v8", "write_v4_cs", "write_bulk"))
     res["read_only_gbs"] = max(res["read_v4_gbs"], res["read_v8_gbs"])
     res["copy_gbs"] = max(res["copy_v4_gbs"], res["copy_v8_gbs"])

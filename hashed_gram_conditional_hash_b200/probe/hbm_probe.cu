@@ -11,7 +11,8 @@
 //   3 write, cp.async.bulk from a 32 KB shared tile (the bulk-copy engine)
 //   4 read, 16-byte ld.global.nc          5 read, 32-byte ld.global.nc.v8
 //   6 copy, 16-byte                        7 copy, 32-byte
-// and engram_probe_gather: random 128-byte rows out of a large source.
+// and engram_probe_gather: random 128-byte rows out of a large source;
+// engram_probe_fma: the fp32 multiply-add rate, packed pairs or scalar.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -146,7 +147,49 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(char* dst, const char*
   }
 }
 
+// fp32 multiply-add rate: 16 independent chains per thread of fma(x, acc, y),
+// as eight packed pairs (__ffma2_rn) or sixteen scalar fmaf; iters steps
+// each; one float per thread keeps the chains live.
+template <bool PACKED>
+__global__ void __launch_bounds__(256) fma_chain_kernel(float* out, int iters, float a, float b) {
+  float r = 0.f;
+  if (PACKED) {
+    float2 acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = make_float2(threadIdx.x * 0.001f + i, i * 0.5f);
+    const float2 x = make_float2(a, b), y = make_float2(b, a);
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = __ffma2_rn(x, acc[i], y);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r += acc[i].x + acc[i].y;
+  } else {
+    float acc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = threadIdx.x * 0.001f + i;
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = fmaf((i & 1) ? b : a, acc[i], (i & 1) ? a : b);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r += acc[i];
+  }
+  out[static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x] = r;
+}
+
 }  // namespace
+
+// Runs fma_chain_kernel (packed != 0: __ffma2_rn pairs, else scalar fmaf) with
+// blocks x 256 threads, iters steps of 16 multiply-adds per thread; out holds
+// blocks * 256 floats.  Returns a cudaError_t.
+extern "C" int engram_probe_fma(int packed, float* out, int blocks, int iters, void* stream) {
+  if (out == nullptr || blocks <= 0 || iters <= 0) return static_cast<int>(cudaErrorInvalidValue);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (packed) fma_chain_kernel<true><<<blocks, 256, 0, s>>>(out, iters, 0.999f, 0.001f);
+  else fma_chain_kernel<false><<<blocks, 256, 0, s>>>(out, iters, 0.999f, 0.001f);
+  return static_cast<int>(cudaGetLastError());
+}
 
 // Gathers out_bytes / 128 rows of 128 bytes from a source of src_bytes (both
 // multiples of 128, pointers 32-byte aligned) at pseudo-random row indices;
