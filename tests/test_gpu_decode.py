@@ -82,7 +82,7 @@ def test_chunked_prefill_with_state(chunks):
 
 
 @pytest.mark.parametrize("B,hc,hidden,dil,orders", [(9, 1, 512, 3, (2, 3)), (17, 4, 768, 2, (2,)),
-                                                     (8, 3, 256, 5, (2, 3, 5))])
+                                                     (8, 3, 256, 5, (2, 3, 5)), (5, 2, 256, 8, (1, 8))])
 def test_decode_steps_partial_blocks_and_branch_counts(B, hc, hidden, dil, orders):
     # every token a decode step (T = 1 with the state): batches that leave the
     # decode conv's last block of sequences partly empty, one to four branches,

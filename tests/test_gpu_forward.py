@@ -53,6 +53,8 @@ SMALL = [
     dict(B=2, T=60, raw_vocab=6500),                              # raw ids through the lookup
     dict(B=2, T=41, row_dim=32),                                  # 64-byte rows (generic gather)
     dict(B=1, T=37, row_dim=128, orders=(2, 3, 4)),               # 256-byte rows (generic gather)
+    dict(B=2, T=33, orders=(2,), heads_per_order=1),               # one head in all (16-row gather)
+    dict(B=2, T=40, orders=(1, 8), dilation=8),                    # a unigram and the largest order
 ]
 
 
